@@ -1,0 +1,33 @@
+"""Reference oracle for the MiMo-V2-Flash hybrid attention operator.
+
+TEST INFRASTRUCTURE ONLY.  This package is a plain, slow, float64 CPU
+restatement of what the operator computes, written from the MiMo-V2-Flash
+model documentation (Transformers model doc, "Key features: hybrid attention"
+bullet and the ``MiMoV2FlashConfig`` parameter list).  Only the test suite,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it.  The CUDA library never calls it and
+shares no code, constant table or helper with it.
+
+Modules
+-------
+``attention``  vectorised fp64 prefill and decode (NumPy matmuls per query block).
+``brute``      scalar triple loops for tiny shapes, used to pin ``attention``.
+
+Every function here is pinned by a ``-m "not gpu"`` test against something
+other than itself (brute force, closed forms, a library special case, or the
+constants the documentation prints).  One choice is *not* pinned by the
+pages: the exact sink formula.  The documentation names a "learnable attention
+sink bias" but prints no formula; the reading used here (one logit per query
+head added as ``exp(sink)`` to the softmax normaliser, no value vector, not
+multiplied by the softmax scale) is a stated reading, so parity of the sink
+term is "parity unpinned" with respect to the original model and pinned only
+with respect to that reading.
+"""
+
+from .attention import (  # noqa: F401
+    DEFAULT_SCALE_DQK,
+    decode,
+    prefill,
+    ring_slot_position,
+    visible,
+)
