@@ -1,0 +1,164 @@
+"""Python binding of the MiMo-V2-Flash hybrid attention library (sm_100a).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libmimo_attn.so`` (C ABI in ``include/mimo_attn.h``).  PyTorch is
+used for device memory and the current stream.  There is no fallback: if the
+library cannot be loaded, importing this package raises.
+
+Entry points (same names as the C ABI):
+
+* ``mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, ...)``
+* ``mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, ...)``
+* ``mimo_attn_decode_workspace_size(...)``, ``mimo_attn_device_status(...)``
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmimo_attn.so")
+
+MIMO_OK = 0
+MIMO_ERR_INVALID_ARG = 1
+MIMO_ERR_UNSUPPORTED = 2
+MIMO_ERR_CUDA = 3
+MIMO_ERR_WORKSPACE = 4
+MIMO_ERR_TIMEOUT = 5
+MIMO_DTYPE_BF16 = 0
+MIMO_DTYPE_F32 = 1
+
+#: entry points declared in include/mimo_attn.h
+EXPORTED = (
+    "mimo_attn_prefill",
+    "mimo_attn_decode_workspace_size",
+    "mimo_attn_decode",
+    "mimo_attn_last_error",
+    "mimo_attn_device_status",
+)
+
+
+class MimoAttnError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"mimo_attn status {status}: {msg}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [
+        ("num_heads_q", ctypes.c_int),
+        ("num_heads_kv", ctypes.c_int),
+        ("head_dim_qk", ctypes.c_int),
+        ("head_dim_v", ctypes.c_int),
+        ("softmax_scale", ctypes.c_float),
+        ("v_scale", ctypes.c_float),
+        ("out_dtype", ctypes.c_int),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with global_attention_swa_b200._build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    dp = ctypes.POINTER(Dims)
+    lib.mimo_attn_prefill.argtypes = [dp, vp, vp, vp, vp, i32, vp, i32, i32, i32, vp, vp, vp]
+    lib.mimo_attn_prefill.restype = i32
+    lib.mimo_attn_decode_workspace_size.argtypes = [dp, i32, i32, i32]
+    lib.mimo_attn_decode_workspace_size.restype = sz
+    lib.mimo_attn_decode.argtypes = [dp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]
+    lib.mimo_attn_decode.restype = i32
+    lib.mimo_attn_last_error.argtypes = []
+    lib.mimo_attn_last_error.restype = ctypes.c_char_p
+    lib.mimo_attn_device_status.argtypes = [vp]
+    lib.mimo_attn_device_status.restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def _check(status):
+    if status != MIMO_OK:
+        raise MimoAttnError(status, lib.mimo_attn_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_dims(hq, hkv, dqk=192, dv=128, softmax_scale=None, v_scale=1.0, out_dtype=torch.bfloat16):
+    return Dims(hq, hkv, dqk, dv,
+                0.0 if softmax_scale is None else float(softmax_scale),
+                float(v_scale),
+                MIMO_DTYPE_F32 if out_dtype == torch.float32 else MIMO_DTYPE_BF16)
+
+
+def mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, out=None, lse=None,
+                      out_dtype=torch.bfloat16, softmax_scale=None, v_scale=1.0,
+                      return_lse=True, stream=None):
+    """Packed varlen prefill.  q [Nt,Hq,192], k [Nt,Hkv,192], v [Nt,Hkv,128] bf16 (CUDA).
+
+    Returns (out [Nt,Hq,128], lse [Hq,Nt] fp32 or None).
+    """
+    nt, hq, dqk = q.shape
+    hkv, dv = k.shape[1], v.shape[2]
+    if out is None:
+        out = torch.empty((nt, hq, dv), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((hq, nt), dtype=torch.float32, device=q.device)
+    dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
+    _check(lib.mimo_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks),
+                                 int(window), _ptr(cu_seqlens), int(cu_seqlens.numel() - 1), nt,
+                                 int(max_seqlen), _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def mimo_attn_decode_workspace_size(hq, hkv, batch, capacity, window, dqk=192, dv=128):
+    dims = make_dims(hq, hkv, dqk, dv)
+    return int(lib.mimo_attn_decode_workspace_size(ctypes.byref(dims), batch, capacity, window))
+
+
+def mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, out=None, lse=None,
+                     workspace=None, out_dtype=torch.bfloat16, softmax_scale=None, v_scale=1.0,
+                     return_lse=True, stream=None):
+    """One decode step.  q [B,Hq,192]; caches [B,C,Hkv,192/128] bf16; seqlens [B] int32.
+
+    Returns (out [B,Hq,128], lse [B,Hq] fp32 or None).
+    """
+    B, hq, dqk = q.shape
+    C, hkv = k_cache.shape[1], k_cache.shape[2]
+    dv = v_cache.shape[3]
+    if out is None:
+        out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
+    need = int(lib.mimo_attn_decode_workspace_size(ctypes.byref(dims), B, C, int(window)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(seqlens), B, C, int(window), _ptr(sinks), _ptr(out),
+                                _ptr(lse), _ptr(workspace), wbytes, _stream(stream)))
+    return out, lse
+
+
+def mimo_attn_device_status(stream=None):
+    """Synchronise the stream; raise if a kernel recorded a device-side error."""
+    _check(lib.mimo_attn_device_status(_stream(stream)))
+
+
+def default_scale(dqk=192):
+    return 1.0 / math.sqrt(dqk)

@@ -1,0 +1,386 @@
+// Decode: one query token per sequence against a KV cache (global linear
+// cache or sliding-window ring), split over the key axis.
+//
+// MiMo-V2-Flash model doc: MiMoV2FlashModel.forward, `past_key_values` (only
+// the new token is fed after the first call) and the "Key features" hybrid
+// attention bullet (SWA layers keep only the window; the learnable sink).
+//
+// Work unit = (sequence b, key/value head g, split c).  The G <= 16 query heads
+// that share head g are packed as the M = 16 rows of a warp-level
+// mma.sync.m16n8k16 (bf16 in, fp32 accumulate): the 16 heads read every K/V
+// byte once, which is what makes this step HBM-bound rather than bound by
+// scalar FMA throughput (16 flop per cache byte).
+//
+// Pipeline per CTA: warp 4 streams 64-key K/V tiles (K: 3 boxes of 64 dims,
+// V: 2 boxes, 128-byte swizzle) into a ring of kStages shared-memory stages
+// with TMA; warps 0-3 each take 16 keys of every tile, compute scores,
+// update an online softmax in base 2 and accumulate P.V in registers.  The
+// four warps merge at the end.  With one split the sink is folded in and the
+// result written out; otherwise (o, m, l) partials go to the workspace and
+// decode_combine_kernel merges them with the sink.
+#pragma once
+
+#include "common.cuh"
+
+namespace mimo {
+
+constexpr int kDecTileKeys = 64;
+constexpr int kDecStages = 4;
+constexpr int kDecKBytes = kDecTileKeys * 192 * 2;   // 24576
+constexpr int kDecVBytes = kDecTileKeys * 128 * 2;   // 16384
+constexpr int kDecStageBytes = kDecKBytes + kDecVBytes;
+constexpr int kDecThreads = 160;                     // 4 consumer warps + 1 producer warp
+constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 /*align*/ + 128 /*barriers*/;
+
+struct DecodeParams {
+  const __nv_bfloat16* q;  // [B, Hq, 192]
+  const int32_t* seqlens;  // [B]
+  const float* sinks;      // [Hq] or null
+  void* out;               // [B, Hq, 128]
+  float* lse;              // [B, Hq] or null
+  float* ws_o;             // [B*Hkv*nsplit, 16, 128]
+  float* ws_ml;            // [B*Hkv*nsplit, 16, 2]
+  int B, C, Hq, Hkv, G;
+  int window;
+  int ring;     // 1: ring cache (C == window)
+  int chunk;    // keys per split, multiple of 64
+  int nsplit;   // splits per (b, g)
+  float scale_log2;  // softmax_scale * log2(e)
+  float v_scale;
+  int out_f32;
+};
+
+// Visible slot range [lo, hi) of sequence b (see mimo_attn.h).
+__device__ __forceinline__ void decode_range(const DecodeParams& p, int L, int& lo, int& hi) {
+  if (L < 0) {
+    record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    L = 0;
+  }
+  if (p.ring) {
+    lo = 0;
+    hi = min(L, p.C);
+  } else {
+    if (L > p.C) {
+      record_status(1 /* MIMO_ERR_INVALID_ARG */);
+      L = p.C;
+    }
+    hi = L;
+    lo = p.window > 0 ? max(0, L - p.window) : 0;
+  }
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  extern __shared__ __align__(1024) uint8_t dsmem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * kDecStageBytes);
+  uint64_t* empty = full + kDecStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int lo, hi;
+  decode_range(p, p.seqlens[b], lo, hi);
+  const int s0 = lo + split * p.chunk;
+  const int s1 = min(hi, s0 + p.chunk);
+  if (p.nsplit > 1 && s0 >= s1) return;  // empty split: the combine skips it
+  if (timed_out_before()) return;
+  const int nkeys = max(0, s1 - s0);
+  const int ntiles = (nkeys + kDecTileKeys - 1) / kDecTileKeys;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int row0 = b * p.C + s0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int st = t % kDecStages;
+        if (t >= kDecStages) {
+          if (!wait_bounded(&empty[st], ((t / kDecStages) - 1) & 1, abort_flag)) break;
+        }
+        uint8_t* kb = smem + st * kDecStageBytes;
+        uint8_t* vb = kb + kDecKBytes;
+        mbar_arrive_expect_tx(&full[st], kDecStageBytes);
+        const int y = row0 + t * kDecTileKeys;
+#pragma unroll
+        for (int c = 0; c < 3; ++c) tma_load_2d(kb + c * 8192, &tm_k, &full[st], g * 192 + c * 64, y);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) tma_load_2d(vb + c * 8192, &tm_v, &full[st], g * 128 + c * 64, y);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int r0 = lane >> 2;        // rows (heads) r0 and r0 + 8
+    const int cq = (lane & 3) * 2;   // column pair within an 8-wide block
+    // Q fragments for all 12 k-steps of 16 dims; rows >= G are zero.
+    uint32_t qa[12][4];
+    {
+      const int h0 = g * p.G + r0, h1 = g * p.G + r0 + 8;
+      const bool v0 = r0 < p.G, v1 = r0 + 8 < p.G;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (v0 ? h0 : 0)) * 192);
+      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (v1 ? h1 : 0)) * 192);
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk) {
+        const int d = kk * 16 + cq;
+        qa[kk][0] = v0 ? __ldg(q0 + d / 2) : 0u;
+        qa[kk][1] = v1 ? __ldg(q1 + d / 2) : 0u;
+        qa[kk][2] = v0 ? __ldg(q0 + (d + 8) / 2) : 0u;
+        qa[kk][3] = v1 ? __ldg(q1 + (d + 8) / 2) : 0u;
+      }
+    }
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY;  // running max (base 2) for rows r0, r0+8
+    float l0 = 0.f, l1 = 0.f;              // per-thread partial sums
+
+    const int kw = warp * 16;  // this warp's 16 keys within each tile
+    const uint32_t sbase = smem_u32(smem);
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % kDecStages;
+      if (!wait_bounded(&full[st], (t / kDecStages) & 1, abort_flag)) break;
+      const int valid = min(kDecTileKeys, nkeys - t * kDecTileKeys);
+      if (kw < valid) {
+        const uint32_t kb = sbase + st * kDecStageBytes;
+        const uint32_t vb = kb + kDecKBytes;
+        // ---- S = Q K^T for keys kw .. kw+15 (two n-blocks of 8)
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+          // ldmatrix.x4 rows: lanes 0-7 keys kw+0..7 dims +0; 8-15 keys kw+0..7 dims +8;
+          // 16-23 keys kw+8..15 dims +0; 24-31 keys kw+8..15 dims +8.
+          const int krow = kw + (lane & 7) + ((lane >> 4) << 3);
+          const int kcol = ((lane >> 3) & 1) * 8;
+#pragma unroll
+          for (int kk = 0; kk < 12; ++kk) {
+            const int c = kk >> 2;                       // 64-dim box
+            const int col = (kk & 3) * 16 + kcol;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + c * 8192 + sw128_offset(krow, col), b0, b1, b2, b3);
+            mma_bf16_16816(s[0], qa[kk], b0, b1);
+            mma_bf16_16816(s[1], qa[kk], b2, b3);
+          }
+        }
+        // ---- scale to base 2 and mask keys past the split's end
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = kw + n * 8 + cq + e;
+            const bool ok = key < valid;
+            s[n][e] = ok ? s[n][e] * p.scale_log2 : -INFINITY;
+            s[n][2 + e] = ok ? s[n][2 + e] * p.scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, s[n][e]);
+            mx1 = fmaxf(mx1, s[n][2 + e]);
+          }
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        // mn is finite: this warp has at least one valid key in the tile
+        const float a0 = ex2(m0 - mn0), a1 = ex2(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        uint32_t pa[4];
+        {
+          float p00 = ex2(s[0][0] - mn0), p01 = ex2(s[0][1] - mn0);
+          float p02 = ex2(s[0][2] - mn1), p03 = ex2(s[0][3] - mn1);
+          float p10 = ex2(s[1][0] - mn0), p11 = ex2(s[1][1] - mn0);
+          float p12 = ex2(s[1][2] - mn1), p13 = ex2(s[1][3] - mn1);
+          l0 = l0 * a0 + (p00 + p01 + p10 + p11);
+          l1 = l1 * a1 + (p02 + p03 + p12 + p13);
+          pa[0] = pack_bf16(p00, p01);
+          pa[1] = pack_bf16(p02, p03);
+          pa[2] = pack_bf16(p10, p11);
+          pa[3] = pack_bf16(p12, p13);
+        }
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          o[n][0] *= a0;
+          o[n][1] *= a0;
+          o[n][2] *= a1;
+          o[n][3] *= a1;
+        }
+        // ---- O += P V.  ldmatrix.trans rows: lanes 0-7 keys kw+0..7, 8-15 keys kw+8..15
+        // (dims +0), 16-23 keys kw+0..7, 24-31 keys kw+8..15 (dims +8).
+        const int vrow = kw + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int vcol = (lane >> 4) * 8;
+        const bool partial = (kw + 16 > valid);
+        // keys held by this thread in the V fragments: kw+cq+{0,1} (b0) and kw+8+cq+{0,1} (b1)
+        const uint32_t mk0 = (kw + cq < valid ? 0x0000FFFFu : 0u) | (kw + cq + 1 < valid ? 0xFFFF0000u : 0u);
+        const uint32_t mk1 = (kw + 8 + cq < valid ? 0x0000FFFFu : 0u) | (kw + 9 + cq < valid ? 0xFFFF0000u : 0u);
+#pragma unroll
+        for (int n2 = 0; n2 < 8; ++n2) {
+          const int c = n2 >> 2;  // 64-dim box
+          const int col = (n2 & 3) * 16 + vcol;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vb + c * 8192 + sw128_offset(vrow, col), b0, b1, b2, b3);
+          if (partial) {  // invalid slots may hold anything: zero them
+            b0 &= mk0; b1 &= mk1; b2 &= mk0; b3 &= mk1;
+          }
+          mma_bf16_16816(o[2 * n2], pa, b0, b1);
+          mma_bf16_16816(o[2 * n2 + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    // ---- reduce l over the quad; merge the 4 warps through shared memory
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // all consumers done with the stages
+    float* so = reinterpret_cast<float*>(smem);      // [4 warps][16 rows][128]
+    float* sm = so + 4 * 16 * 128;                   // [4][16] max
+    float* sl = sm + 4 * 16;                         // [4][16] sum
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      const int col = n * 8 + cq;
+      so[(warp * 16 + r0) * 128 + col] = o[n][0];
+      so[(warp * 16 + r0) * 128 + col + 1] = o[n][1];
+      so[(warp * 16 + r0 + 8) * 128 + col] = o[n][2];
+      so[(warp * 16 + r0 + 8) * 128 + col + 1] = o[n][3];
+    }
+    if ((lane & 3) == 0) {
+      sm[warp * 16 + r0] = m0;
+      sm[warp * 16 + r0 + 8] = m1;
+      sl[warp * 16 + r0] = l0;
+      sl[warp * 16 + r0 + 8] = l1;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // 128 threads: thread -> (row = tid / 8, 16 columns)
+    const int tid = threadIdx.x;
+    const int row = tid >> 3;
+    const int c0 = (tid & 7) * 16;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 16 + row]);
+    float wgt[4];
+    float Ls = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      wgt[w] = (M == -INFINITY) ? 0.f : ex2(sm[w * 16 + row] - M);
+      Ls += wgt[w] * sl[w * 16 + row];
+    }
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) a += wgt[w] * so[(w * 16 + row) * 128 + c0 + e];
+      acc[e] = a;
+    }
+    if (row < p.G) {
+      const int h = g * p.G + row;
+      if (p.nsplit == 1) {
+        // fold the sink: it joins the normaliser only
+        const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
+        const float Mf = fmaxf(M, sg);
+        float scl = 0.f, Lf = 0.f;
+        if (Mf != -INFINITY) {
+          scl = (M == -INFINITY) ? 0.f : ex2(M - Mf);
+          Lf = Ls * scl + ((sg == -INFINITY) ? 0.f : ex2(sg - Mf));
+        }
+        const float f = (Lf > 0.f) ? p.v_scale * scl / Lf : 0.f;
+        const size_t ob = ((size_t)b * p.Hq + h) * 128 + c0;
+        if (p.out_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_float4(acc[4 * e] * f, acc[4 * e + 1] * f, acc[4 * e + 2] * f, acc[4 * e + 3] * f);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            uint4 u;
+            u.x = pack_bf16(acc[8 * e + 0] * f, acc[8 * e + 1] * f);
+            u.y = pack_bf16(acc[8 * e + 2] * f, acc[8 * e + 3] * f);
+            u.z = pack_bf16(acc[8 * e + 4] * f, acc[8 * e + 5] * f);
+            u.w = pack_bf16(acc[8 * e + 6] * f, acc[8 * e + 7] * f);
+            dst[e] = u;
+          }
+        }
+        if (p.lse && (tid & 7) == 0)
+          p.lse[(size_t)b * p.Hq + h] = (Lf > 0.f) ? (Mf * 0.6931471805599453f + logf(Lf)) : -INFINITY;
+      } else {
+        const size_t unit = ((size_t)b * p.Hkv + g) * p.nsplit + split;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + (unit * 16 + row) * 128 + c0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+        if ((tid & 7) == 0) {
+          p.ws_ml[(unit * 16 + row) * 2 + 0] = M;
+          p.ws_ml[(unit * 16 + row) * 2 + 1] = Ls;
+        }
+      }
+    }
+  }
+}
+
+// Merge the split partials of every (b, query head) and fold the sink:
+//   M = max(sigma, max_c m_c),  Z = 2^(sigma-M) + sum_c 2^(m_c-M) l_c,
+//   out = v_scale * sum_c 2^(m_c-M) o_c / Z,   lse = ln Z + M ln 2.
+// One warp per (b, h); lane handles 4 of the 128 value columns.
+__global__ void __launch_bounds__(256)
+    decode_combine_kernel(const DecodeParams p) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= p.B * p.Hq) return;
+  const int b = wid / p.Hq, h = wid % p.Hq;
+  const int g = h / p.G, row = h % p.G;
+  int lo, hi;
+  decode_range(p, p.seqlens[b], lo, hi);
+  const int nused = min(p.nsplit, max(0, (hi - lo + p.chunk - 1) / p.chunk));
+  const size_t unit0 = ((size_t)b * p.Hkv + g) * p.nsplit;
+  const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
+  float M = sg;
+  for (int c = 0; c < nused; ++c) M = fmaxf(M, p.ws_ml[((unit0 + c) * 16 + row) * 2]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float Z = 0.f;
+  if (M != -INFINITY) {
+    Z = (sg == -INFINITY) ? 0.f : ex2(sg - M);
+    for (int c = 0; c < nused; ++c) {
+      const float mc = p.ws_ml[((unit0 + c) * 16 + row) * 2];
+      const float lc = p.ws_ml[((unit0 + c) * 16 + row) * 2 + 1];
+      const float w = (mc == -INFINITY) ? 0.f : ex2(mc - M);
+      Z += w * lc;
+      const float4 oc = reinterpret_cast<const float4*>(p.ws_o + ((unit0 + c) * 16 + row) * 128)[lane];
+      acc.x += w * oc.x;
+      acc.y += w * oc.y;
+      acc.z += w * oc.z;
+      acc.w += w * oc.w;
+    }
+  }
+  const float f = (Z > 0.f) ? p.v_scale / Z : 0.f;
+  const size_t ob = ((size_t)b * p.Hq + h) * 128 + lane * 4;
+  if (p.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob) =
+        make_float4(acc.x * f, acc.y * f, acc.z * f, acc.w * f);
+  } else {
+    uint2 u;
+    u.x = pack_bf16(acc.x * f, acc.y * f);
+    u.y = pack_bf16(acc.z * f, acc.w * f);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob) = u;
+  }
+  if (p.lse && lane == 0)
+    p.lse[(size_t)b * p.Hq + h] = (Z > 0.f) ? (M * 0.6931471805599453f + logf(Z)) : -INFINITY;
+}
+
+}  // namespace mimo

@@ -1,0 +1,346 @@
+// Host side of the C ABI declared in include/mimo_attn.h: argument checks,
+// TMA descriptor encoding, the decode split plan, and kernel launches.
+// All kernels of the library live in this one translation unit so that the
+// device status word is shared without relocatable device code.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mimo_attn.h"
+#include "common.cuh"
+#include "decode_kernel.cuh"
+#include "prefill_kernel.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+mimo_status_t fail(mimo_status_t st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+mimo_status_t fail(mimo_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+mimo_status_t ok() {
+  g_last_error.clear();
+  return MIMO_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- tensor maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor with `rank` dims (innermost first), byte strides of dims 1.., box sizes.
+mimo_status_t make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MIMO_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bd[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bd[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bd,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MIMO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MIMO_OK;
+}
+
+// ---------------------------------------------------------------- common checks
+
+mimo_status_t check_dims(const mimo_attn_dims_t* d) {
+  if (!d) return fail(MIMO_ERR_INVALID_ARG, "dims is NULL");
+  if (d->num_heads_q <= 0 || d->num_heads_kv <= 0)
+    return fail(MIMO_ERR_INVALID_ARG, "head counts must be positive (Hq=%d, Hkv=%d)",
+                d->num_heads_q, d->num_heads_kv);
+  if (d->num_heads_q % d->num_heads_kv)
+    return fail(MIMO_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", d->num_heads_q,
+                d->num_heads_kv);
+  if (d->head_dim_qk != 192 || d->head_dim_v != 128)
+    return fail(MIMO_ERR_UNSUPPORTED, "only head_dim_qk=192, head_dim_v=128 are built (got %d, %d)",
+                d->head_dim_qk, d->head_dim_v);
+  if (d->out_dtype != MIMO_DTYPE_BF16 && d->out_dtype != MIMO_DTYPE_F32)
+    return fail(MIMO_ERR_INVALID_ARG, "out_dtype must be MIMO_DTYPE_BF16 or MIMO_DTYPE_F32");
+  if (!std::isfinite(d->softmax_scale) || !std::isfinite(d->v_scale))
+    return fail(MIMO_ERR_INVALID_ARG, "softmax_scale and v_scale must be finite");
+  return MIMO_OK;
+}
+
+float scale_log2_of(const mimo_attn_dims_t* d) {
+  const float s = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / std::sqrt((float)d->head_dim_qk);
+  return s * 1.4426950408889634f;
+}
+
+float v_scale_of(const mimo_attn_dims_t* d) { return d->v_scale != 0.f ? d->v_scale : 1.0f; }
+
+mimo_status_t cuda_check(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(MIMO_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MIMO_OK;
+}
+
+// Opt every kernel into its dynamic shared memory once per device.
+mimo_status_t ensure_attributes() {
+  static std::mutex mu;
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(MIMO_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(mu);
+  if (done[dev]) return MIMO_OK;
+  mimo_status_t st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::prefill_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kPfSmemBytes),
+                       "prefill smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kDecSmemBytes),
+                       "decode smem attribute")))
+    return st;
+  done[dev] = true;
+  return MIMO_OK;
+}
+
+// ---------------------------------------------------------------- decode plan
+
+struct DecodePlan {
+  int ring, cap_eff, chunk, nsplit;
+};
+
+int env_chunk() {
+  static int v = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const char* s = std::getenv("MIMO_DECODE_CHUNK");
+    v = s ? std::atoi(s) : 0;
+  });
+  return v;
+}
+
+DecodePlan decode_plan(int batch, int hkv, int capacity, int window) {
+  DecodePlan pl;
+  pl.ring = (window > 0 && capacity == window) ? 1 : 0;
+  pl.cap_eff = (!pl.ring && window > 0) ? std::min(window, capacity) : capacity;
+  const int tile = mimo::kDecTileKeys;
+  // Aim for >= 2 resident work units per SM across the grid, splits of
+  // 256..2048 keys; a single split needs no workspace and no combine.
+  int chunk = env_chunk();
+  if (chunk <= 0) {
+    const long units = (long)batch * hkv;
+    const long want = 2L * 148;
+    long nsplit = (want + units - 1) / units;
+    long max_split = std::max(1L, ((long)pl.cap_eff + 255) / 256);
+    nsplit = std::max(1L, std::min(nsplit, max_split));
+    long c = ((long)pl.cap_eff + nsplit - 1) / nsplit;
+    chunk = (int)std::min<long>(c, 2048);
+  }
+  chunk = std::max(tile, ((chunk + tile - 1) / tile) * tile);
+  pl.chunk = chunk;
+  pl.nsplit = std::max(1, (pl.cap_eff + chunk - 1) / chunk);
+  return pl;
+}
+
+size_t workspace_bytes_of(int batch, int hkv, const DecodePlan& pl) {
+  if (pl.nsplit <= 1) return 0;
+  const size_t units = (size_t)batch * hkv * pl.nsplit;
+  return units * 16 * 128 * sizeof(float) + units * 16 * 2 * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mimo_attn_last_error(void) { return g_last_error.c_str(); }
+
+mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, const void* k,
+                                const void* v, const float* sinks, int window,
+                                const int32_t* cu_seqlens, int num_seqs, int total_tokens,
+                                int max_seqlen, void* out, float* lse, void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  if (window < 0) return fail(MIMO_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0)
+    return fail(MIMO_ERR_INVALID_ARG, "sizes must be non-negative");
+  if (!cu_seqlens) return fail(MIMO_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (total_tokens == 0 || num_seqs == 0 || max_seqlen == 0) return ok();  // nothing to do
+  if (!q || !k || !v || !out) return fail(MIMO_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && ((uintptr_t)lse & 3u)) || (sinks && ((uintptr_t)sinks & 3u)))
+    return fail(MIMO_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned");
+  if (max_seqlen > total_tokens)
+    return fail(MIMO_ERR_INVALID_ARG, "max_seqlen (%d) > total_tokens (%d)", max_seqlen, total_tokens);
+  if (num_seqs > 65535) return fail(MIMO_ERR_UNSUPPORTED, "num_seqs > 65535");
+  const int Hq = dims->num_heads_q, Hkv = dims->num_heads_kv, G = Hq / Hkv;
+  if ((st = ensure_attributes())) return st;
+
+  CUtensorMap tq, tk, tv;
+  {
+    const uint64_t d[3] = {192, (uint64_t)Hq, (uint64_t)total_tokens};
+    const uint64_t s[2] = {192 * 2, (uint64_t)Hq * 192 * 2};
+    const uint32_t b[3] = {64, 1, 128};
+    if ((st = make_map(&tq, q, 3, d, s, b))) return st;
+  }
+  {
+    const uint64_t d[3] = {192, (uint64_t)Hkv, (uint64_t)total_tokens};
+    const uint64_t s[2] = {192 * 2, (uint64_t)Hkv * 192 * 2};
+    const uint32_t b[3] = {64, 1, 128};
+    if ((st = make_map(&tk, k, 3, d, s, b))) return st;
+  }
+  {
+    const uint64_t d[3] = {128, (uint64_t)Hkv, (uint64_t)total_tokens};
+    const uint64_t s[2] = {128 * 2, (uint64_t)Hkv * 128 * 2};
+    const uint32_t b[3] = {64, 1, 128};
+    if ((st = make_map(&tv, v, 3, d, s, b))) return st;
+  }
+  mimo::PrefillParams p;
+  p.cu_seqlens = cu_seqlens;
+  p.sinks = sinks;
+  p.out = out;
+  p.lse = lse;
+  p.total = total_tokens;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.pairs_per_group = (G + 1) / 2;
+  p.scale_log2 = scale_log2_of(dims);
+  p.v_scale = v_scale_of(dims);
+  p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+  const int qtiles = (max_seqlen + mimo::kPfTile - 1) / mimo::kPfTile;
+  dim3 grid(qtiles, Hkv * p.pairs_per_group, num_seqs);
+  mimo::prefill_kernel<<<grid, mimo::kPfThreads, mimo::kPfSmemBytes, (cudaStream_t)stream>>>(
+      tq, tk, tv, p);
+  if ((st = cuda_check(cudaGetLastError(), "prefill launch"))) return st;
+  return ok();
+}
+
+size_t mimo_attn_decode_workspace_size(const mimo_attn_dims_t* dims, int batch, int capacity,
+                                       int window) {
+  if (!dims || dims->num_heads_kv <= 0 || batch <= 0 || capacity <= 0 || window < 0) return 0;
+  return workspace_bytes_of(batch, dims->num_heads_kv,
+                            decode_plan(batch, dims->num_heads_kv, capacity, window));
+}
+
+mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* seqlens, int batch,
+                               int capacity, int window, const float* sinks, void* out,
+                               float* lse, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  if (window < 0) return fail(MIMO_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if (batch < 0 || capacity < 0) return fail(MIMO_ERR_INVALID_ARG, "sizes must be non-negative");
+  if (batch == 0) return ok();
+  if (capacity == 0) return fail(MIMO_ERR_INVALID_ARG, "capacity must be positive");
+  if (!q || !k_cache || !v_cache || !seqlens || !out)
+    return fail(MIMO_ERR_INVALID_ARG, "q, k_cache, v_cache, seqlens and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (lse && ((uintptr_t)lse & 3u)) || (sinks && ((uintptr_t)sinks & 3u)))
+    return fail(MIMO_ERR_INVALID_ARG, "q, caches and out must be 16-byte aligned");
+  const int Hq = dims->num_heads_q, Hkv = dims->num_heads_kv, G = Hq / Hkv;
+  if (G > 16) return fail(MIMO_ERR_UNSUPPORTED, "decode packs at most 16 query heads per KV head (got %d)", G);
+  if ((long)batch * capacity > 0x7fffffffL)
+    return fail(MIMO_ERR_UNSUPPORTED, "batch * capacity must fit in int32");
+  if (batch > 65535 || Hkv > 65535) return fail(MIMO_ERR_UNSUPPORTED, "batch or Hkv > 65535");
+  const DecodePlan pl = decode_plan(batch, Hkv, capacity, window);
+  const size_t need = workspace_bytes_of(batch, Hkv, pl);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(MIMO_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+  if (need > 0 && !aligned16(workspace))
+    return fail(MIMO_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((st = ensure_attributes())) return st;
+
+  CUtensorMap tk, tv;
+  {
+    const uint64_t d[2] = {(uint64_t)Hkv * 192, (uint64_t)batch * capacity};
+    const uint64_t s[1] = {(uint64_t)Hkv * 192 * 2};
+    const uint32_t b[2] = {64, (uint32_t)mimo::kDecTileKeys};
+    if ((st = make_map(&tk, k_cache, 2, d, s, b))) return st;
+  }
+  {
+    const uint64_t d[2] = {(uint64_t)Hkv * 128, (uint64_t)batch * capacity};
+    const uint64_t s[1] = {(uint64_t)Hkv * 128 * 2};
+    const uint32_t b[2] = {64, (uint32_t)mimo::kDecTileKeys};
+    if ((st = make_map(&tv, v_cache, 2, d, s, b))) return st;
+  }
+  mimo::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.seqlens = seqlens;
+  p.sinks = sinks;
+  p.out = out;
+  p.lse = lse;
+  const size_t units = (size_t)batch * Hkv * pl.nsplit;
+  p.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+  p.ws_ml = need ? static_cast<float*>(workspace) + units * 16 * 128 : nullptr;
+  p.B = batch;
+  p.C = capacity;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.ring = pl.ring;
+  p.chunk = pl.chunk;
+  p.nsplit = pl.nsplit;
+  p.scale_log2 = scale_log2_of(dims);
+  p.v_scale = v_scale_of(dims);
+  p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+  dim3 grid(pl.nsplit, Hkv, batch);
+  mimo::decode_split_kernel<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, (cudaStream_t)stream>>>(
+      tk, tv, p);
+  if ((st = cuda_check(cudaGetLastError(), "decode launch"))) return st;
+  if (pl.nsplit > 1) {
+    const int warps = batch * Hq;
+    const int blocks = (warps * 32 + 255) / 256;
+    mimo::decode_combine_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(p);
+    if ((st = cuda_check(cudaGetLastError(), "decode combine launch"))) return st;
+  }
+  return ok();
+}
+
+mimo_status_t mimo_attn_device_status(void* stream) {
+  mimo_status_t st;
+  if ((st = cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize"))) return st;
+  int v = 0;
+  if ((st = cuda_check(cudaMemcpyFromSymbol(&v, mimo::g_device_status, sizeof(int)), "read status")))
+    return st;
+  const int zero = 0;
+  if ((st = cuda_check(cudaMemcpyToSymbol(mimo::g_device_status, &zero, sizeof(int)), "clear status")))
+    return st;
+  if (v == 0) return ok();
+  return fail(static_cast<mimo_status_t>(v), "device status %d recorded by a kernel", v);
+}
+
+}  // extern "C"

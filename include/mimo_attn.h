@@ -1,0 +1,153 @@
+/*
+ * mimo_attn.h -- C ABI of the MiMo-V2-Flash hybrid attention operator for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the operator computes (MiMo-V2-Flash model doc, "Key features":
+ * hybrid attention bullet; MiMoV2FlashConfig parameters num_attention_heads,
+ * num_key_value_heads, head_dim, v_head_dim, sliding_window):
+ *
+ *   causal grouped-query attention, Hq query heads over Hkv key/value heads
+ *   (query head h reads key/value head h / (Hq/Hkv)), query/key dim Dqk and
+ *   value dim Dv, softmax scale s (default 1/sqrt(Dqk)), an optional sliding
+ *   window, and a per-query-head attention-sink logit sigma_h:
+ *
+ *     visible(i, j)  <=>  0 <= i - j  and  (window == 0 or i - j <= window-1)
+ *     S_j  = s * <q_i, k_j>                         over visible j
+ *     m    = max(sigma_h, max_j S_j)
+ *     Z    = exp(sigma_h - m) + sum_j exp(S_j - m)
+ *     out  = v_scale * sum_j exp(S_j - m) v_j / Z   (the sink has no value)
+ *     lse  = m + ln Z                                (natural log, with sink)
+ *
+ *   window = 129 is the model's sliding-window layer (the query plus the
+ *   previous 128 keys); window = 0 is its global layer.  Layers interleave
+ *   5 sliding-window : 1 global; the caller passes the layer's window.
+ *   The sink formula is this library's reading: the documentation names a
+ *   "learnable attention sink bias" but prints no formula.
+ *
+ * Conventions for every entry point
+ *   - Supported shapes: Dqk == 192, Dv == 128, Hq % Hkv == 0, Hq/Hkv <= 16
+ *     for decode; other shapes return MIMO_ERR_UNSUPPORTED.
+ *   - All tensor arguments are caller-owned DEVICE pointers, contiguous,
+ *     16-byte aligned.  The library keeps no pointer after the call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  No host synchronisation happens.
+ *     The return status covers argument validation and launch errors;
+ *     a fault inside a kernel surfaces at the caller's next synchronisation.
+ *   - Every wait inside a kernel is bounded.  A wait that gives up records
+ *     MIMO_ERR_TIMEOUT in a device status word, which
+ *     mimo_attn_device_status() reads and clears.
+ *   - On a non-OK status, mimo_attn_last_error() returns a message for the
+ *     calling thread.
+ */
+#ifndef MIMO_ATTN_H_
+#define MIMO_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MIMO_OK = 0,
+  MIMO_ERR_INVALID_ARG = 1,   /* NULL pointer, negative size, bad window ... */
+  MIMO_ERR_UNSUPPORTED = 2,   /* head dims other than 192/128, group > 16 ... */
+  MIMO_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  MIMO_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than required */
+  MIMO_ERR_TIMEOUT = 5        /* a bounded in-kernel wait gave up */
+} mimo_status_t;
+
+typedef enum { MIMO_DTYPE_BF16 = 0, MIMO_DTYPE_F32 = 1 } mimo_dtype_t;
+
+typedef struct {
+  int num_heads_q;     /* Hq  (64 in the model) */
+  int num_heads_kv;    /* Hkv (4 in the model)  */
+  int head_dim_qk;     /* Dqk (192) */
+  int head_dim_v;      /* Dv  (128) */
+  float softmax_scale; /* <= 0 selects 1/sqrt(Dqk) */
+  float v_scale;       /* output multiplier (attention_value_scale); 0 selects 1 */
+  int out_dtype;       /* mimo_dtype_t of `out` */
+} mimo_attn_dims_t;
+
+/*
+ * Packed variable-length prefill (one attention layer over all prompt tokens).
+ *
+ *   q          [total_tokens, Hq,  Dqk] bf16, post-RoPE
+ *   k          [total_tokens, Hkv, Dqk] bf16, post-RoPE
+ *   v          [total_tokens, Hkv, Dv ] bf16
+ *   sinks      [Hq] fp32 sink logits (natural-log units), or NULL for none
+ *   window     0 = global causal; >= 1 = the query plus window-1 earlier keys
+ *   cu_seqlens [num_seqs + 1] int32 on the device: cu[0] = 0, non-decreasing,
+ *              cu[num_seqs] = total_tokens.  Sequence s owns tokens
+ *              [cu[s], cu[s+1]); lengths of 0 are allowed.
+ *   max_seqlen >= every sequence length (sizes the launch; not read back)
+ *   out        [total_tokens, Hq, Dv] in dims->out_dtype
+ *   lse        [Hq, total_tokens] fp32, or NULL to skip
+ *
+ * Work is split over (sequence, 128-query tile, pair of query heads of one
+ * key/value group).  Key tiles wholly outside the window are never loaded.
+ */
+mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims,
+                                const void* q, const void* k, const void* v,
+                                const float* sinks, int window,
+                                const int32_t* cu_seqlens, int num_seqs,
+                                int total_tokens, int max_seqlen,
+                                void* out, float* lse, void* stream);
+
+/*
+ * Bytes of device workspace mimo_attn_decode needs for these sizes
+ * (split-KV partial results).  0 when one split covers every sequence.
+ */
+size_t mimo_attn_decode_workspace_size(const mimo_attn_dims_t* dims, int batch,
+                                       int capacity, int window);
+
+/*
+ * One decode step: one query token per sequence against its KV cache
+ * (MiMoV2FlashModel.forward, past_key_values: only the new token is fed).
+ *
+ *   q          [batch, Hq, Dqk] bf16, post-RoPE
+ *   k_cache    [batch, capacity, Hkv, Dqk] bf16
+ *   v_cache    [batch, capacity, Hkv, Dv ] bf16
+ *   seqlens    [batch] int32 on the device: tokens so far INCLUDING the
+ *              current one, whose K/V are already in the cache; the query
+ *              sits at position L-1.
+ *   window     0 = global.  If window > 0 and capacity == window the cache is
+ *              a RING: token p lives in slot p mod capacity and every slot
+ *              below min(L, capacity) is visible.  Otherwise the cache is
+ *              LINEAR (slot = position) and requires L <= capacity; slots
+ *              [max(0, L-window), L) are visible (all of [0, L) if window=0).
+ *              L > capacity on a linear cache is clamped to capacity and
+ *              recorded as MIMO_ERR_INVALID_ARG in the device status word.
+ *   sinks      [Hq] fp32 or NULL
+ *   out        [batch, Hq, Dv] in dims->out_dtype
+ *   lse        [batch, Hq] fp32 or NULL
+ *   workspace  device scratch of at least mimo_attn_decode_workspace_size()
+ *              bytes (may be NULL when that size is 0).  Calls sharing one
+ *              workspace must not overlap on the GPU.
+ *
+ * Slots past a sequence's length are never read into the result (their
+ * contents may be anything, NaN included).
+ */
+mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q,
+                               const void* k_cache, const void* v_cache,
+                               const int32_t* seqlens, int batch, int capacity,
+                               int window, const float* sinks, void* out,
+                               float* lse, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+const char* mimo_attn_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that
+ * bounded in-kernel waits and device-side argument checks write.  Returns
+ * MIMO_OK, MIMO_ERR_TIMEOUT, MIMO_ERR_INVALID_ARG or MIMO_ERR_CUDA.
+ */
+mimo_status_t mimo_attn_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMO_ATTN_H_ */

@@ -137,9 +137,9 @@ def prefill(q, k, v, sinks, window, cu_seqlens, scale=None, v_scale=1.0,
     """
     if window < 0:
         raise ValueError("window must be >= 0")
-    Q, K, Vv = _f64(q), _f64(k), _f64(v)
+    K, Vv = _f64(k), _f64(v)
     cu = _i64(cu_seqlens)
-    Nt, Hq, Dqk = Q.shape
+    Nt, Hq, Dqk = q.shape
     Hkv, Dv = K.shape[1], Vv.shape[2]
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
@@ -148,7 +148,17 @@ def prefill(q, k, v, sinks, window, cu_seqlens, scale=None, v_scale=1.0,
         scale = 1.0 / math.sqrt(Dqk)
     sig = np.full(Hq, -np.inf) if sinks is None else _f64(sinks).reshape(Hq)
 
-    rows = np.arange(Nt) if rows is None else _i64(rows).reshape(-1)
+    if rows is None:
+        rows = np.arange(Nt)
+        Q = _f64(q)                       # [n, Hq, Dqk], row t = token t
+    else:
+        rows = _i64(rows).reshape(-1)
+        if hasattr(q, "detach"):
+            import torch
+
+            Q = _f64(q[torch.as_tensor(rows, device=q.device)])
+        else:
+            Q = _f64(np.asarray(q)[rows])
     n = rows.shape[0]
     out = np.zeros((n, Hq, Dv))
     lse = np.full((Hq, n), -np.inf)
@@ -168,7 +178,7 @@ def prefill(q, k, v, sinks, window, cu_seqlens, scale=None, v_scale=1.0,
     def run(job):
         sel, qpos, b0, b1, h, kpos = job
         g = h // G
-        o, l = _one_head(Q[rows[sel], h, :], K[b0:b1, g, :], Vv[b0:b1, g, :],
+        o, l = _one_head(Q[sel, h, :], K[b0:b1, g, :], Vv[b0:b1, g, :],
                          qpos, kpos, window, sig[h], scale)
         return sel, h, o, l
 

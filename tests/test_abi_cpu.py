@@ -1,0 +1,95 @@
+"""The C-ABI library loads, exports what include/*.h declares, and validates
+arguments on the host.  CPU only: no call here reaches a kernel launch."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import global_attention_swa_b200 as mimo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # a 16-byte aligned non-null address; never dereferenced (validation fails first)
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(mimo_attn_\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    assert set(mimo.EXPORTED) <= declared_symbols()
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(mimo.LIB_PATH)
+    for name in sorted(declared_symbols()):
+        assert hasattr(lib, name), name
+
+
+def _dims(hq=64, hkv=4, dqk=192, dv=128):
+    return mimo.make_dims(hq, hkv, dqk, dv)
+
+
+def _prefill(dims, q=FAKE, k=FAKE, v=FAKE, window=129, cu=FAKE, nseq=1, total=128, maxlen=128,
+             out=FAKE):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    d = ctypes.byref(dims) if dims is not None else None
+    return mimo.lib.mimo_attn_prefill(d, p(q), p(k), p(v), None, window, p(cu), nseq, total,
+                                      maxlen, p(out), None, None)
+
+
+def test_prefill_rejects_bad_arguments():
+    assert _prefill(None) == mimo.MIMO_ERR_INVALID_ARG
+    assert _prefill(_dims(), window=-1) == mimo.MIMO_ERR_INVALID_ARG
+    assert _prefill(_dims(hq=6, hkv=4)) == mimo.MIMO_ERR_INVALID_ARG
+    assert _prefill(_dims(dqk=128)) == mimo.MIMO_ERR_UNSUPPORTED
+    assert _prefill(_dims(dv=192)) == mimo.MIMO_ERR_UNSUPPORTED
+    assert _prefill(_dims(), q=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _prefill(_dims(), cu=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _prefill(_dims(), k=FAKE + 2) == mimo.MIMO_ERR_INVALID_ARG   # misaligned
+    assert _prefill(_dims(), maxlen=129, total=128) == mimo.MIMO_ERR_INVALID_ARG
+
+
+def test_prefill_empty_is_a_no_op():
+    assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
+    assert _prefill(_dims(), nseq=0, total=0, maxlen=0) == mimo.MIMO_OK
+
+
+def _decode(dims, batch=2, cap=1024, window=0, ws=None, ws_bytes=0, q=FAKE, out=FAKE):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    return mimo.lib.mimo_attn_decode(ctypes.byref(dims), p(q), p(FAKE), p(FAKE), p(FAKE), batch,
+                                     cap, window, None, p(out), None, p(ws), ws_bytes, None)
+
+
+def test_decode_rejects_bad_arguments():
+    assert _decode(_dims(), window=-3) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode(_dims(), q=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode(_dims(), out=FAKE + 4) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode(_dims(hq=64, hkv=2)) == mimo.MIMO_ERR_UNSUPPORTED   # 32 heads per group
+    assert _decode(_dims(), cap=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode(_dims(), batch=0) == mimo.MIMO_OK
+
+
+def test_decode_workspace_contract():
+    need = mimo.mimo_attn_decode_workspace_size(64, 4, 64, 262144, 0)
+    assert need > 0 and need % 16 == 0
+    assert _decode(_dims(), batch=64, cap=262144, ws=None) == mimo.MIMO_ERR_WORKSPACE
+    assert _decode(_dims(), batch=64, cap=262144, ws=FAKE, ws_bytes=need - 16) == mimo.MIMO_ERR_WORKSPACE
+    assert "workspace" in mimo.lib.mimo_attn_last_error().decode()
+
+
+def test_ring_decode_needs_no_workspace():
+    # a 129-slot ring with window 129 is covered by one split per (sequence, KV head)
+    assert mimo.mimo_attn_decode_workspace_size(64, 4, 64, 129, 129) == 0
+
+
+def test_last_error_is_empty_after_success():
+    assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
+    assert mimo.lib.mimo_attn_last_error().decode() == ""
