@@ -1,0 +1,465 @@
+"""Benchmark of the MiMo-V2-Flash hybrid attention hot path on B200.
+
+One step = one pass over every kernel of the path at the model's head shape
+(64 query heads, 4 key/value heads, head dims 192 / 128), seeded synthetic
+bf16 inputs ~N(0, 1), fp32 sink logits ~N(0, 1):
+
+  1. sliding-window prefill, T = 32768, window 129      (HBM-bound)
+  2. global prefill, T = 32768, causal                   (tensor-core-bound)
+  3. global decode, batch 64, lengths ~U[1024, 262144] in 262144-slot caches
+     (split-KV + combine; HBM-bound)
+  4. sliding-window decode, batch 64, 129-slot ring caches (latency-bound)
+
+Reported value: the step's roofline floor (sum over the four kernels of
+max(useful FLOP / bf16 tensor peak, algorithmic bytes / HBM peak), peaks from
+MEASURED_PEAKS.json) divided by the measured step time, in % -- summed over
+GPUs for N > 1 (each GPU runs its own step: weak scaling, no collective on the
+data path).  Per-kernel TFLOP/s and GB/s are in "parts".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode KV-cache GB/s, % of B200 roofline"
+UNIT = "% of B200 roofline (sum over GPUs)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+T_PREFILL = 32768
+SWA = W.SWA_WINDOW
+HQ, HKV, DQK, DV = W.HQ, W.HKV, W.DQK, W.DV
+FLOP_PER_PAIR = 2 * DQK + 2 * DV          # per (visible pair, query head)
+KV_BYTES_PER_TOKEN = HKV * (DQK + DV) * 2   # 2560 B of K and V per cached token
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- work model
+
+def visible_pairs(T, window):
+    if window == 0:
+        return T * (T + 1) // 2
+    w = window
+    return sum(min(i + 1, w) for i in range(T)) if T < 4096 else (
+        w * (w + 1) // 2 + (T - w) * w if T >= w else T * (T + 1) // 2)
+
+
+def prefill_work(T, window):
+    flops = FLOP_PER_PAIR * HQ * visible_pairs(T, window)
+    byts = T * (HQ * DQK * 2 + HKV * (DQK + DV) * 2 + HQ * DV * 2 + HQ * 4)
+    return flops, byts
+
+
+def decode_work(lengths, window, capacity):
+    ring = window > 0 and capacity == window
+    vis = [min(L, capacity) if ring else (min(L, window) if window > 0 else L) for L in lengths]
+    flops = FLOP_PER_PAIR * HQ * sum(vis)
+    byts = sum(vis) * KV_BYTES_PER_TOKEN + len(lengths) * HQ * (DQK * 2 + DV * 2 + 4)
+    return flops, byts
+
+
+def floor_s(flops, byts, peaks):
+    return max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(1.0)  # let nvidia-smi start sampling before the timed region
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), max=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        load = [r for r in rows if r["power"] > 300] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, peaks, peak_kind):
+    import global_attention_swa_b200 as mimo
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    seed = 1000 * rank
+    # --- inputs resident in HBM
+    swa = W.prefill_inputs([T_PREFILL], seed=seed + 1, device=dev)
+    ga = W.prefill_inputs([T_PREFILL], seed=seed + 2, device=dev)
+    lengths = W.decode_b64_lengths(0)
+    dga = W.decode_inputs(lengths, W.DECODE_GA_CAPACITY, 0, seed=seed + 3, device=dev)
+    dsw = W.decode_inputs(lengths, SWA, SWA, seed=seed + 4, device=dev)
+    o_swa = torch.empty((T_PREFILL, HQ, DV), dtype=torch.bfloat16, device=dev)
+    o_ga = torch.empty_like(o_swa)
+    l_swa = torch.empty((HQ, T_PREFILL), dtype=torch.float32, device=dev)
+    l_ga = torch.empty_like(l_swa)
+    o_dga = torch.empty((64, HQ, DV), dtype=torch.bfloat16, device=dev)
+    o_dsw = torch.empty_like(o_dga)
+    l_dga = torch.empty((64, HQ), dtype=torch.float32, device=dev)
+    l_dsw = torch.empty_like(l_dga)
+    ws_ga = torch.empty(max(1, mimo.mimo_attn_decode_workspace_size(
+        HQ, HKV, 64, W.DECODE_GA_CAPACITY, 0)), dtype=torch.uint8, device=dev)
+    ws_sw = torch.empty(max(1, mimo.mimo_attn_decode_workspace_size(HQ, HKV, 64, SWA, SWA)),
+                        dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        rec = (lambda i: evs[i].record(stream)) if evs else (lambda i: None)
+        rec(0)
+        mimo.mimo_attn_prefill(swa.q, swa.k, swa.v, swa.sinks, SWA, swa.cu_seqlens, T_PREFILL,
+                               out=o_swa, lse=l_swa)
+        rec(1)
+        mimo.mimo_attn_prefill(ga.q, ga.k, ga.v, ga.sinks, 0, ga.cu_seqlens, T_PREFILL,
+                               out=o_ga, lse=l_ga)
+        rec(2)
+        mimo.mimo_attn_decode(dga.q, dga.k_cache, dga.v_cache, dga.seqlens, 0, dga.sinks,
+                              out=o_dga, lse=l_dga, workspace=ws_ga)
+        rec(3)
+        mimo.mimo_attn_decode(dsw.q, dsw.k_cache, dsw.v_cache, dsw.seqlens, SWA, dsw.sinks,
+                              out=o_dsw, lse=l_dsw, workspace=ws_sw)
+        rec(4)
+
+    launches_per_step = 2 + (2 if ws_ga.numel() > 1 else 1) + (2 if ws_sw.numel() > 1 else 1)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    mimo.mimo_attn_device_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        t_wall = time.perf_counter()
+        for k in range(args.steps):
+            flush.zero_()          # L2 flush between steps (outside the events)
+            step(evs[k])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    mimo.mimo_attn_device_status()
+
+    per = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(4)]
+                    for k in range(args.steps)])  # ms [K, 4]
+    step_ms = per.sum(axis=1)
+    mean_ms = float(step_ms.mean())
+    if world > 1:
+        t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        max_ms = float(t.item())
+    else:
+        max_ms = mean_ms
+
+    works = [prefill_work(T_PREFILL, SWA), prefill_work(T_PREFILL, 0),
+             decode_work(lengths, 0, W.DECODE_GA_CAPACITY), decode_work(lengths, SWA, SWA)]
+    floors = [floor_s(f, b, peaks) for f, b in works]
+    floor_step_ms = 1e3 * sum(floors)
+    value = 100.0 * world * floor_step_ms / max_ms
+    names = ["prefill_swa_T32768_W129", "prefill_global_T32768", "decode_global_B64_cap262144",
+             "decode_swa_ring_B64_W129"]
+    bounds = ["hbm", "tensor", "hbm", "hbm"]
+    parts = {}
+    for i, n in enumerate(names):
+        ms = float(per[:, i].mean())
+        f, b = works[i]
+        parts[n] = {"ms": round(ms, 4), "TFLOP/s": round(f / (ms * 1e-3) / 1e12, 2),
+                    "GB/s": round(b / (ms * 1e-3) / 1e9, 1),
+                    "roofline_frac": round(1e3 * floors[i] / ms, 4), "bound": bounds[i],
+                    "useful_flop": f, "algorithmic_bytes": b}
+
+    # dominant kernel: global prefill (tensor-bound)
+    ga_ms = float(per[:, 1].mean())
+    ga_tflops = works[1][0] / (ga_ms * 1e-3) / 1e12
+    roofline = {"kernel": "prefill_kernel (global, T=32768)", "bound": "tensor",
+                "achieved": round(ga_tflops, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(ga_tflops / peaks["bf16_tflops"], 4),
+                "peak_kind": f"{peak_kind} burst bf16",
+                "frac_of_sustained": round(ga_tflops / peaks["bf16_tflops_sustained"], 4),
+                "traffic": None}
+    tr = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr):
+        roofline["traffic"] = json.load(open(tr)).get("prefill_global_T32768")
+
+    # --- e2e through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, mimo, swa, ga, dga, dsw, lengths, dev, floor_step_ms, world,
+                      o_swa, o_ga, o_dga, o_dsw, l_swa, l_ga, l_dga, l_dsw, ws_ga, ws_sw)
+
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, N(0,1) fp32 sinks)",
+        "config": {"workload": "hybrid attention step at model head shape: SWA prefill "
+                               "T=32768 W=129 + global prefill T=32768 + decode B=64 (global, "
+                               "262144-slot caches, lengths ~U[1024,262144]) + decode B=64 "
+                               "(129-slot SWA ring)",
+                   "heads_q": HQ, "heads_kv": HKV, "head_dim_qk": DQK, "head_dim_v": DV,
+                   "seq_len": T_PREFILL, "decode_batch": 64, "parallelism": f"replicas{world}",
+                   "l2": "flushed between steps (256 MB write); every input > L2 except the "
+                         "21 MB ring caches",
+                   "floor_ms_per_step": round(floor_step_ms, 4),
+                   "peaks": {**peaks, "source": peak_kind}},
+        "parts": parts,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "wall_s_timed_region": round(t_wall, 4),
+    }
+    return res
+
+
+def run_e2e(args, mimo, swa, ga, dga, dsw, lengths, dev, floor_step_ms, world,
+            o_swa, o_ga, o_dga, o_dsw, l_swa, l_ga, l_dga, l_dsw, ws_ga, ws_sw):
+    """Same step through the public API, inputs copied from pinned host memory each
+    step and every output read back.  KV caches are the decode layers' persistent
+    state and stay resident; the decode step's input is the new query."""
+    host = {}
+    for name, t in (("sq", swa.q), ("sk", swa.k), ("sv", swa.v), ("gq", ga.q), ("gk", ga.k),
+                    ("gv", ga.v), ("dq", dga.q), ("rq", dsw.q)):
+        host[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        host[name].copy_(t)
+    outs = {}
+    for name, t in (("o_swa", o_swa), ("o_ga", o_ga), ("o_dga", o_dga), ("o_dsw", o_dsw),
+                    ("l_swa", l_swa), ("l_ga", l_ga), ("l_dga", l_dga), ("l_dsw", l_dsw)):
+        outs[name] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    dq = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for k in host:
+            dq[k].copy_(host[k], non_blocking=True)
+        mimo.mimo_attn_prefill(dq["sq"], dq["sk"], dq["sv"], swa.sinks, SWA, swa.cu_seqlens,
+                               T_PREFILL, out=o_swa, lse=l_swa)
+        mimo.mimo_attn_prefill(dq["gq"], dq["gk"], dq["gv"], ga.sinks, 0, ga.cu_seqlens,
+                               T_PREFILL, out=o_ga, lse=l_ga)
+        mimo.mimo_attn_decode(dq["dq"], dga.k_cache, dga.v_cache, dga.seqlens, 0, dga.sinks,
+                              out=o_dga, lse=l_dga, workspace=ws_ga)
+        mimo.mimo_attn_decode(dq["rq"], dsw.k_cache, dsw.v_cache, dsw.seqlens, SWA, dsw.sinks,
+                              out=o_dsw, lse=l_dsw, workspace=ws_sw)
+        for k, t in (("o_swa", o_swa), ("o_ga", o_ga), ("o_dga", o_dga), ("o_dsw", o_dsw),
+                     ("l_swa", l_swa), ("l_ga", l_ga), ("l_dga", l_dga), ("l_dsw", l_dsw)):
+            outs[k].copy_(t, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(100.0 * world * floor_step_ms / ms, 3), "unit": UNIT,
+            "ms_per_step": round(ms, 3), "steps": n,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- oracle arms
+
+class OracleSample:
+    """The fp64 oracle on a bounded sample of one step (inputs generated once)."""
+
+    def __init__(self, rows_swa, rows_ga, decode_seqs):
+        self.rows_swa, self.rows_ga, self.decode_seqs = rows_swa, rows_ga, decode_seqs
+        self.pre = {SWA: W.prefill_inputs([T_PREFILL], seed=1), 0: W.prefill_inputs([T_PREFILL], seed=2)}
+        lengths = W.decode_b64_lengths(0)
+        self.Ls = [lengths[b] for b in range(decode_seqs)]
+        self.dec = [(0, None, W.decode_inputs(self.Ls, max(self.Ls), 0, seed=3, poison=False)),
+                    (SWA, SWA, W.decode_inputs(self.Ls, SWA, SWA, seed=4, poison=False))]
+        self.sample = (
+            f"{rows_swa} random query rows x 64 heads of the T=32768 SWA prefill, {rows_ga} of "
+            f"the global prefill, {decode_seqs} of the 64 global-decode sequences and "
+            f"{decode_seqs} ring-decode sequence(s); value = roofline floor of the sampled "
+            f"work / oracle seconds")
+
+    def run(self, peaks, seed=0):
+        import oracle
+
+        t_total = 0.0
+        floor_sample = 0.0
+        # prefills: random query rows (all 64 heads); the sampled share of pairs / bytes
+        for window, nrows in ((SWA, self.rows_swa), (0, self.rows_ga)):
+            x = self.pre[window]
+            rows = np.sort(np.random.default_rng(seed * 7 + window).choice(
+                T_PREFILL, nrows, replace=False))
+            t0 = time.perf_counter()
+            oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, rows=rows)
+            t_total += time.perf_counter() - t0
+            pairs = sum(min(int(r) + 1, window) if window else int(r) + 1 for r in rows)
+            f = FLOP_PER_PAIR * HQ * pairs
+            b = prefill_work(T_PREFILL, window)[1] * nrows / T_PREFILL
+            floor_sample += floor_s(f, b, peaks)
+        for window, cap, d in self.dec:
+            c = d.capacity
+            t0 = time.perf_counter()
+            oracle.decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks,
+                          ring=(cap is not None))
+            t_total += time.perf_counter() - t0
+            f, b = decode_work(self.Ls, window, c)
+            floor_sample += floor_s(f, b, peaks)
+        return 100.0 * floor_sample / t_total, t_total
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, peaks, peak_kind):
+    vals, secs = [], []
+    smp = OracleSample(rows_swa=64, rows_ga=8, decode_seqs=1)
+    sample = smp.sample
+    for i in range(args.warmup + args.steps):
+        v, s = smp.run(peaks, seed=i)
+        if i >= args.warmup:
+            vals.append(v)
+            secs.append(s)
+    v = float(np.mean(vals))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(secs)), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, N(0,1) fp32 sinks)",
+        "config": {"workload": "hybrid attention step at model head shape (bounded sample per "
+                               "step, see cpu_baseline.sample)", "peaks": {**peaks, "source": peak_kind}},
+        "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": cpu_cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks, peak_kind = load_peaks()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, peaks, peak_kind)), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    res = run_ours(args, rank, world, peaks, peak_kind)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(rows_swa=256, rows_ga=24, decode_seqs=1)
+        v, s = smp.run(peaks)
+        res["cpu_baseline"] = {"value": round(v, 6), "unit": UNIT, "cores": cpu_cores(),
+                               "kind": "oracle", "sample": smp.sample, "seconds": round(s, 2)}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

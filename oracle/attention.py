@@ -62,6 +62,17 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
+def _blas_threads(n):
+    try:
+        from threadpoolctl import threadpool_limits
+
+        return threadpool_limits(limits=n, user_api="blas")
+    except Exception:  # pragma: no cover - threadpoolctl missing
+        import contextlib
+
+        return contextlib.nullcontext()
+
+
 def _i64(x):
     if hasattr(x, "detach"):
         return x.detach().cpu().numpy().astype(np.int64)
@@ -98,23 +109,36 @@ def _softmax_with_sink(S, sigma):
     return W, lse
 
 
+def _row_blocks(qpos_sorted):
+    """Runs of sorted query positions spanning fewer than _ROW_BLOCK positions."""
+    n = len(qpos_sorted)
+    start = 0
+    for i in range(1, n + 1):
+        if (i == n or qpos_sorted[i] - qpos_sorted[start] >= _ROW_BLOCK
+                or i - start >= _ROW_BLOCK):
+            yield start, i
+            start = i
+
+
 def _one_head(q_h, K, V, qpos, kpos, window, sigma, scale):
     """All requested query rows of one head against one sequence's keys."""
     n = q_h.shape[0]
     out = np.zeros((n, V.shape[1]))
     lse = np.full(n, -np.inf)
-    for r0 in range(0, n, _ROW_BLOCK):
-        r1 = min(n, r0 + _ROW_BLOCK)
-        ip = qpos[r0:r1]
+    order = np.argsort(qpos, kind="stable")
+    qs = qpos[order]
+    for r0, r1 in _row_blocks(qs):
+        idx = order[r0:r1]
+        ip = qs[r0:r1]
         # keys that can be visible to any row of the block
         lo = 0 if window == 0 else max(0, int(ip.min()) - window + 1)
         hi = int(ip.max()) + 1
         kp = kpos[lo:hi]
-        S = scale * (q_h[r0:r1] @ K[lo:hi].T)
+        S = scale * (q_h[idx] @ K[lo:hi].T)
         S = np.where(visible(ip[:, None], kp[None, :], window), S, -np.inf)
         Wt, l = _softmax_with_sink(S, sigma)
-        out[r0:r1] = Wt @ V[lo:hi]
-        lse[r0:r1] = l
+        out[idx] = Wt @ V[lo:hi]
+        lse[idx] = l
     return out, lse
 
 
@@ -183,7 +207,8 @@ def prefill(q, k, v, sinks, window, cu_seqlens, scale=None, v_scale=1.0,
         return sel, h, o, l
 
     nthreads = threads or len(os.sched_getaffinity(0))
-    with ThreadPoolExecutor(max_workers=nthreads) as ex:
+    # one BLAS thread per worker: the pool over (sequence, head) jobs uses the cores
+    with _blas_threads(1), ThreadPoolExecutor(max_workers=nthreads) as ex:
         for sel, h, o, l in ex.map(run, jobs):
             out[sel, h, :] = o * v_scale
             lse[h, sel] = l

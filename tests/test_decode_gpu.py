@@ -99,8 +99,12 @@ def test_ring_matches_linear_window():
     b, lb = mimo.mimo_attn_decode(q, x.k[None].cuda(), x.v[None].cuda(), sl, 129, x.sinks.cuda(),
                                   out_dtype=torch.float32)
     torch.cuda.synchronize()
-    assert (a - b).abs().max().item() < 1e-5
-    assert (la - lb).abs().max().item() < 1e-5
+    # same keys, different order and split tiling: P is rounded to bf16 against
+    # different running maxima, so the two agree to bf16 precision, not bitwise
+    assert (a - b).abs().max().item() < 2e-3
+    assert (la - lb).abs().max().item() < 1e-4
+    ro, rl = oracle.decode(x.q[L - 1:L], x.k[None], x.v[None], [L], 129, x.sinks, ring=False)
+    P.strict(a, ro, la, rl, what="ring")
 
 
 def test_full_size_decode_global_and_ring():
