@@ -39,6 +39,7 @@ EXPORTED = (
     "mimo_attn_decode",
     "mimo_attn_last_error",
     "mimo_attn_device_status",
+    "mimo_attn_decode_noalloc",
 )
 
 
@@ -81,6 +82,11 @@ def _load():
 
 
 lib = _load()
+
+if hasattr(lib, "mimo_attn_decode_noalloc"):
+    lib.mimo_attn_decode_noalloc.argtypes = [ctypes.POINTER(Dims)] + [ctypes.c_void_p] * 4 + [
+        ctypes.c_int, ctypes.c_int, ctypes.c_int] + [ctypes.c_void_p] * 4
+    lib.mimo_attn_decode_noalloc.restype = ctypes.c_int
 
 
 def _check(status):
@@ -162,3 +168,18 @@ def mimo_attn_device_status(stream=None):
 
 def default_scale(dqk=192):
     return 1.0 / math.sqrt(dqk)
+
+
+def mimo_attn_decode_noalloc(q, k_cache, v_cache, seqlens, window, sinks, out, lse=None,
+                             softmax_scale=None, v_scale=1.0, stream=None):
+    """Decode through the entry point that allocates nothing (see include/mimo_attn.h).
+
+    The caller passes preallocated ``out`` [B,Hq,128] and optional ``lse`` [B,Hq].
+    """
+    B, hq, dqk = q.shape
+    C, hkv = k_cache.shape[1], k_cache.shape[2]
+    dims = make_dims(hq, hkv, dqk, v_cache.shape[3], softmax_scale, v_scale, out.dtype)
+    _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(seqlens), B, C, int(window), _ptr(sinks), _ptr(out),
+                                        _ptr(lse), _stream(stream)))
+    return out, lse

@@ -344,3 +344,68 @@ mimo_status_t mimo_attn_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without allocation.
+//
+// Some callers cannot call cudaMalloc: code that runs inside a host process
+// whose device memory belongs to another allocator (a serving runtime or a
+// framework's memory pool that forbids raw allocations), and latency-critical
+// loops that cannot afford the implicit device synchronisation cudaMalloc and
+// cudaFree may bring.  For them the split-KV partial results live in this
+// file-scope device array instead of a caller-provided workspace.  Every GPU
+// that loads the library reserves it until the process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in; the real address is looked up once
+// per device, with that device current, and cached.
+void* noalloc_scratch(mimo_status_t* st) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = fail(MIMO_ERR_CUDA, "cudaGetDevice failed");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || !p) {
+      *st = fail(MIMO_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" mimo_status_t mimo_attn_decode_noalloc(const mimo_attn_dims_t* dims, const void* q,
+                                                  const void* k_cache, const void* v_cache,
+                                                  const int32_t* seqlens, int batch, int capacity,
+                                                  int window, const float* sinks, void* out,
+                                                  float* lse, void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  const size_t need = mimo_attn_decode_workspace_size(dims, batch, capacity, window);
+  if (need > kNoAllocScratchBytes)
+    return fail(MIMO_ERR_WORKSPACE,
+                "decode needs %zu bytes of scratch but the built-in scratch holds %zu; use fewer "
+                "sequences or a smaller capacity, or mimo_attn_decode with a workspace",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if (need > 0 && !(scratch = noalloc_scratch(&st))) return st;
+  // The split kernel writes every partial the combine kernel reads, so nothing
+  // in the scratch has to start at zero.
+  return mimo_attn_decode(dims, q, k_cache, v_cache, seqlens, batch, capacity, window, sinks, out,
+                          lse, scratch, need > 0 ? kNoAllocScratchBytes : 0, stream);
+}

@@ -136,6 +136,32 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q,
                                float* lse, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/*
+ * mimo_attn_decode without a workspace and without allocating.  The model
+ * documentation has no counterpart to this call: it exists for callers that
+ * cannot call cudaMalloc -- code running in a process whose device memory is
+ * owned by another allocator (a serving runtime or a framework memory pool),
+ * or latency-critical loops that cannot take the device synchronisation an
+ * allocation may cause.  It allocates nothing and calls no allocating routine.
+ *
+ * Arguments are those of mimo_attn_decode minus the workspace.  The split-KV
+ * partials go to a 16 MiB array compiled into the library (every GPU that
+ * loads the library holds it until exit).  Sizes whose workspace
+ * (mimo_attn_decode_workspace_size) exceeds 16 MiB are rejected with
+ * MIMO_ERR_WORKSPACE before any device work.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the previous call's
+ * contents (nothing in it needs to start at zero): calls that overlap on the
+ * GPU, on any streams, race and corrupt each other's results.
+ */
+mimo_status_t mimo_attn_decode_noalloc(const mimo_attn_dims_t* dims, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* seqlens, int batch, int capacity,
+                                       int window, const float* sinks, void* out,
+                                       float* lse, void* stream);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 const char* mimo_attn_last_error(void);
 
