@@ -418,6 +418,48 @@ def run_reference(args, peaks, peak_kind):
 
 # ---------------------------------------------------------------- main
 
+def run_case(args):
+    """One kernel of the path alone (for profiling): prints a small JSON line."""
+    import global_attention_swa_b200 as mimo
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    T = args.seq_len
+    if args.case.startswith("prefill"):
+        window = SWA if args.case == "prefill_swa" else 0
+        x = W.prefill_inputs([T], seed=1, device=dev)
+        out = torch.empty((T, HQ, DV), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((HQ, T), dtype=torch.float32, device=dev)
+        fn = lambda: mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, T,  # noqa: E731
+                                             out=out, lse=lse)
+        work = prefill_work(T, window)
+    else:
+        lengths = W.decode_b64_lengths(0)
+        window, cap = (0, W.DECODE_GA_CAPACITY) if args.case == "decode_global" else (SWA, SWA)
+        d = W.decode_inputs(lengths, cap, window, seed=3, device=dev)
+        fn = lambda: mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks)  # noqa: E731
+        work = decode_work(lengths, window, cap)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    mimo.mimo_attn_device_status()
+    m = float(np.mean(ms)) if ms else float("nan")
+    f, b = work
+    print(json.dumps({"case": args.case, "seq_len": T, "ms": round(m, 4),
+                      "TFLOP/s": round(f / (m * 1e-3) / 1e12, 1),
+                      "GB/s": round(b / (m * 1e-3) / 1e9, 1)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -426,6 +468,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["step", "prefill_swa", "prefill_global", "decode_global",
+                                       "decode_ring"], default="step",
+                    help="run one kernel alone (profiling); 'step' is the benchmark")
+    ap.add_argument("--seq-len", type=int, default=T_PREFILL, help="prefill length for --case")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -443,6 +489,9 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
     torch.cuda.set_device(local)
+    if args.case != "step":
+        run_case(args)
+        return
     if world > 1:
         import datetime
 

@@ -203,12 +203,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           float p02 = ex2(s[0][2] - mn1), p03 = ex2(s[0][3] - mn1);
           float p10 = ex2(s[1][0] - mn0), p11 = ex2(s[1][1] - mn0);
           float p12 = ex2(s[1][2] - mn1), p13 = ex2(s[1][3] - mn1);
-          l0 = l0 * a0 + (p00 + p01 + p10 + p11);
-          l1 = l1 * a1 + (p02 + p03 + p12 + p13);
           pa[0] = pack_bf16(p00, p01);
           pa[1] = pack_bf16(p02, p03);
           pa[2] = pack_bf16(p10, p11);
           pa[3] = pack_bf16(p12, p13);
+          l0 = l0 * a0 + ((p00 + p01) + (p10 + p11));
+          l1 = l1 * a1 + ((p02 + p03) + (p12 + p13));
         }
 #pragma unroll
         for (int n = 0; n < 16; ++n) {

@@ -14,8 +14,14 @@
 //               also allocates / frees the 512 TMEM columns.
 //   warp 9      MMA issuer (one thread):  S_i = Q_i K^T   (tcgen05, SS)
 //                                         O_i += P_i V    (tcgen05, TS: P from TMEM)
+//   warps 10-11 idle (they complete the third warpgroup)
 //   warps 0-3   softmax + epilogue of head 0 (TMEM lanes 0..127, one row each)
 //   warps 4-7   softmax + epilogue of head 1
+//
+// Registers: launched at 168 per thread (384 threads); the producer/MMA
+// warpgroup gives back down to 80 and the two softmax warpgroups take 208
+// (2*128*208 + 128*80 = 63488 <= 384*168 = 64512; per SM sub-partition
+// 208 + 208 + 80 registers x 32 lanes = 15872 <= 16384).
 //
 // TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512).
 // P_i (bf16, two per 32-bit column) overwrites the first 64 columns of S_i.
@@ -35,7 +41,7 @@
 
 namespace mimo {
 
-constexpr int kPfThreads = 320;
+constexpr int kPfThreads = 384;
 constexpr int kPfTile = 128;
 constexpr int kPfQBytes = 128 * 192 * 2;  // 49152: 3 boxes of [128 rows][64 dims]
 constexpr int kPfKBytes = 128 * 192 * 2;  // 49152
@@ -133,7 +139,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
-
+  if (warp >= 8) {
+    setmaxnreg_dec<80>();
+  }
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -229,8 +237,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
+    setmaxnreg_inc<208>();
     const int i = warp >> 2;  // which head of the pair
     if (i == 0 || has1) {
       const int h = i ? h1 : h0;
@@ -253,23 +262,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_wait_ld();
         const bool full_tile = (kpos0 + kPfTile - 1 <= q0) &&
                                (p.window == 0 || (q0 + kPfTile - 1) - kpos0 <= p.window - 1);
-        float mx = -INFINITY;
+        // Row max of the raw scores (the scale is positive, so it commutes with
+        // max), as 8 independent chains to keep the dependency depth short.
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
         if (full_tile) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            s[c] *= p.scale_log2;
-            mx = fmaxf(mx, s[c]);
-          }
+          for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
         } else {
           const int hi_k = qpos - kpos0;                                  // keys <= hi_k visible
           const int lo_k = p.window > 0 ? qpos - p.window + 1 - kpos0 : -1;  // keys >= lo_k visible
 #pragma unroll
           for (int c = 0; c < 128; ++c) {
-            s[c] = (c <= hi_k && c >= lo_k) ? s[c] * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, s[c]);
+            s[c] = (c <= hi_k && c >= lo_k) ? s[c] : -INFINITY;
+            mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
           }
         }
-        const float m_new = fmaxf(m, mx);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_new = fmaxf(m, mx * p.scale_log2);
         float alpha = 1.f;
         bool rescale_o = false;
         if (m_new - m > kRescaleLog2) {  // false when both are -inf (NaN compare)
@@ -278,20 +290,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           m = m_new;
           rescale_o = (t > 0);
         }
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        float rs = 0.f;
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        // P = 2^(s*scale - m), rounded to bf16 for the PV product; the row sum
+        // keeps the unrounded values so that lse stays exact to fp32.
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(s[64 * half + 2 * c] - m_use);
-            const float p1 = ex2(s[64 * half + 2 * c + 1] - m_use);
-            rs += p0 + p1;
-            pk[c] = pack_bf16(p0, p1);
+            const float2 x = fma2(make_float2(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]), sc2, nm2);
+            const float2 e = make_float2(ex2(x.x), ex2(x.y));
+            pk[c] = pack_bf16(e.x, e.y);
+            acc[c & 3] = add2(acc[c & 3], e);
           }
           tmem_st32(tS + 32 * half, pk);
         }
+        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
+        const float2 a = add2(a01, a23);
+        const float rs = a.x + a.y;
         l += rs;
         // O of the previous tile is complete here: S_i(t) was committed after PV_i(t-1).
         if (__any_sync(0xffffffffu, rescale_o)) {

@@ -107,8 +107,8 @@ def test_rescale_path_with_growing_scores():
     x.k = (x.k.float() * 0.25 + ramp * x.q[:, :1].float().sign()).to(torch.bfloat16)
     out, lse = run_gpu(x, 0, torch.float32)
     ro, rl = oracle.prefill(x.q, x.k, x.v, None, 0, x.cu_seqlens)
-    # Attention here is nearly one-hot: P's bf16 rounding (2^-9 relative) then
-    # shows up as up to 2^-9 |v| in the output, hence the |ref|-relative term.
+    # Attention here is nearly one-hot, so |out| ~ |v|: P's bf16 rounding is
+    # covered by the |ref|-relative term of check().
     P.check(out, ro, lse, rl, what="rescale")
 
 
@@ -145,10 +145,7 @@ def full_size_check(lengths, window, hq=64, hkv=4, seed=0, per_seq_random=64, si
     rows = sample_rows(lengths, window, per_seq_random, seed)
     ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, rows=rows)
     idx = torch.as_tensor(rows, device="cuda")
-    cu = np.cumsum([0] + list(lengths))
-    pos = rows - cu[np.searchsorted(cu, rows, side="right") - 1]
-    nvis = pos + 1 if window == 0 else np.minimum(pos + 1, window)
-    P.tiered(out[idx], ro, nvis, lse[:, idx], rl, what=f"full size W={window}")
+    P.check(out[idx], ro, lse[:, idx], rl, what=f"full size W={window}")
 
 
 def test_full_size_swa_32k():
