@@ -85,6 +85,22 @@ def floor_s(flops, byts, peaks):
     return max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(x, world, device=None):
+    """MAX of a per-rank scalar over all ranks (NCCL on GPUs, gloo on CPU)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def step_value(floor_step_ms, max_ms, world):
+    """Whole-job value: every rank ran one step (weak scaling), timed as the max over ranks."""
+    return 100.0 * world * floor_step_ms / max_ms
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -216,18 +232,13 @@ def run_ours(args, rank, world, peaks, peak_kind):
                     for k in range(args.steps)])  # ms [K, 4]
     step_ms = per.sum(axis=1)
     mean_ms = float(step_ms.mean())
-    if world > 1:
-        t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        max_ms = float(t.item())
-    else:
-        max_ms = mean_ms
+    max_ms = max_over_ranks(mean_ms, world, dev)
 
     works = [prefill_work(T_PREFILL, SWA), prefill_work(T_PREFILL, 0),
              decode_work(lengths, 0, W.DECODE_GA_CAPACITY), decode_work(lengths, SWA, SWA)]
     floors = [floor_s(f, b, peaks) for f, b in works]
     floor_step_ms = 1e3 * sum(floors)
-    value = 100.0 * world * floor_step_ms / max_ms
+    value = step_value(floor_step_ms, max_ms, world)
     names = ["prefill_swa_T32768_W129", "prefill_global_T32768", "decode_global_B64_cap262144",
              "decode_swa_ring_B64_W129"]
     bounds = ["hbm", "tensor", "hbm", "hbm"]
@@ -330,12 +341,8 @@ def run_e2e(args, mimo, swa, ga, dga, dsw, lengths, dev, floor_step_ms, world,
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / n
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(100.0 * world * floor_step_ms / ms, 3), "unit": UNIT,
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+    return {"value": round(step_value(floor_step_ms, ms, world), 3), "unit": UNIT,
             "ms_per_step": round(ms, 3), "steps": n,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
