@@ -87,19 +87,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int s0 = lo + split * p.chunk;
   const int s1 = min(hi, s0 + p.chunk);
   if (p.nsplit > 1 && s0 >= s1) return;  // empty split: the combine skips it
-  if (timed_out_before()) return;
   const int nkeys = max(0, s1 - s0);
-  const int ntiles = (nkeys + kDecTileKeys - 1) / kDecTileKeys;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 4);
     }
-    *abort_flag = 0;
+    // sampled once, so every thread of the CTA sees the same decision
+    *abort_flag = timed_out_before() ? 1 : 0;
     fence_mbar_init();
   }
   __syncthreads();
+  // after a recorded timeout elsewhere, stream nothing (results are void anyway)
+  const int ntiles = *abort_flag ? 0 : (nkeys + kDecTileKeys - 1) / kDecTileKeys;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer

@@ -134,6 +134,19 @@ mimo_status_t ensure_attributes() {
   return MIMO_OK;
 }
 
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!counts[dev]) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+      c = 148;
+    counts[dev] = c;
+  }
+  return counts[dev];
+}
+
 // ---------------------------------------------------------------- decode plan
 
 struct DecodePlan {
@@ -239,8 +252,14 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
   p.scale_log2 = scale_log2_of(dims);
   p.v_scale = v_scale_of(dims);
   p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
-  const int qtiles = (max_seqlen + mimo::kPfTile - 1) / mimo::kPfTile;
-  dim3 grid(qtiles, Hkv * p.pairs_per_group, num_seqs);
+  p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+  p.num_seqs = num_seqs;
+  p.num_qtiles = (max_seqlen + mimo::kPfTile - 1) / mimo::kPfTile;
+  const long items = (long)p.num_qtiles * Hkv * p.pairs_per_group * num_seqs;
+  if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
+  p.num_items = (int)items;
+  // persistent: one CTA per SM (225 KB of shared memory and all of TMEM each)
+  const int grid = (int)std::min<long>(items, sm_count());
   mimo::prefill_kernel<<<grid, mimo::kPfThreads, mimo::kPfSmemBytes, (cudaStream_t)stream>>>(
       tq, tk, tv, p);
   if ((st = cuda_check(cudaGetLastError(), "prefill launch"))) return st;

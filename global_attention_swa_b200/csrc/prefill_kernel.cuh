@@ -6,9 +6,14 @@
 // MiMoV2FlashConfig (64 query heads over 4 key/value heads, head_dim 192 for
 // query/key, v_head_dim 128, sliding_window 129).
 //
-// One CTA = one 128-query tile of one sequence x two query heads of the same
+// Work item = one 128-query tile of one sequence x two query heads of the same
 // key/value group.  Both heads see exactly the same key tiles, so each K/V
 // tile staged in shared memory feeds two 128x128 score tiles.
+//
+// The kernel is persistent: one CTA per SM walks the item list (heaviest
+// query tiles first, snake order across CTAs).  Barrier phases run on across
+// items, so the next item's Q / K loads and first score MMAs overlap the
+// current item's last P.V products and its epilogue.
 //
 //   warp 8      TMA producer: Q (2 x 48 KB), K ring (2 x 48 KB), V (32 KB);
 //               also allocates / frees the 512 TMEM columns.
@@ -19,9 +24,9 @@
 //   warps 4-7   softmax + epilogue of head 1
 //
 // Registers: launched at 168 per thread (384 threads); the producer/MMA
-// warpgroup gives back down to 80 and the two softmax warpgroups take 208
-// (2*128*208 + 128*80 = 63488 <= 384*168 = 64512; per SM sub-partition
-// 208 + 208 + 80 registers x 32 lanes = 15872 <= 16384).
+// warpgroup gives back down to 104 and the two softmax warpgroups take 200
+// (2*128*200 + 128*104 = 64512 = 384*168; per SM sub-partition
+// 200 + 200 + 104 registers x 32 lanes = 16128 <= 16384).
 //
 // TMEM columns: S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512).
 // P_i (bf16, two per 32-bit column) overwrites the first 64 columns of S_i.
@@ -62,9 +67,13 @@ struct PrefillParams {
   int total, Hq, Hkv, G;
   int window;
   int pairs_per_group;        // ceil(G / 2)
+  int num_seqs;
+  int num_qtiles;             // ceil(max_seqlen / 128)
+  int num_items;              // num_qtiles * Hkv * pairs_per_group * num_seqs
   float scale_log2;           // softmax_scale * log2(e)
   float v_scale;
   int out_f32;
+  int out_v8;                 // out is 32-byte aligned: one full sector per store
 };
 
 // K-major operand (rows of 64 bf16 = 128 B, 8-row groups 1024 B apart).
@@ -76,6 +85,44 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
   return smem_desc_sw128(addr, 16384, 1024);
 }
 
+// One work item, decoded.  Items are numbered heaviest query tile first;
+// within a query tile, key/value head pair then sequence.
+struct PfItem {
+  int b0, len, q0, g, h0, j_lo, n_kt;
+  bool has1, valid;
+};
+
+__device__ __forceinline__ int pf_item_index(int round, int cta, int ctas) {
+  return round * ctas + ((round & 1) ? (ctas - 1 - cta) : cta);  // snake order
+}
+
+__device__ __forceinline__ PfItem pf_decode(const PrefillParams& p, int item) {
+  PfItem it;
+  const int per_q = p.Hkv * p.pairs_per_group * p.num_seqs;
+  const int qt = p.num_qtiles - 1 - item / per_q;
+  int rem = item % per_q;
+  const int seq = rem % p.num_seqs;
+  const int pair = rem / p.num_seqs;
+  it.g = pair / p.pairs_per_group;
+  const int pp = pair % p.pairs_per_group;
+  it.h0 = it.g * p.G + 2 * pp;
+  it.has1 = (2 * pp + 1) < p.G;
+  it.b0 = p.cu_seqlens[seq];
+  it.len = p.cu_seqlens[seq + 1] - it.b0;
+  it.q0 = qt * kPfTile;
+  it.valid = it.q0 < it.len;
+  if (it.valid) {
+    const int last_q = min(it.q0 + kPfTile - 1, it.len - 1);
+    const int j_hi = last_q / kPfTile;
+    it.j_lo = p.window > 0 ? max(0, it.q0 - p.window + 1) / kPfTile : 0;
+    it.n_kt = j_hi - it.j_lo + 1;
+  } else {
+    it.j_lo = 0;
+    it.n_kt = 0;
+  }
+  return it;
+}
+
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -84,50 +131,36 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPfOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;
-  uint64_t* v_empty = bars + 6;
-  uint64_t* s_full = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;   // [2]
-  uint64_t* o_full = bars + 11;  // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 14);
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;   // [2]
+  uint64_t* k_empty = bars + 4;  // [2]
+  uint64_t* v_full = bars + 6;
+  uint64_t* v_empty = bars + 7;
+  uint64_t* s_full = bars + 8;   // [2]
+  uint64_t* p_full = bars + 10;  // [2]
+  uint64_t* o_full = bars + 12;  // [2]
+  uint64_t* o_empty = bars + 14; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int seq = blockIdx.z;
-  const int b0 = p.cu_seqlens[seq];
-  const int len = p.cu_seqlens[seq + 1] - b0;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest (last) tiles first
-  const int q0 = qt * kPfTile;
-  if (q0 >= len || timed_out_before()) return;
-  const int g = blockIdx.y / p.pairs_per_group;
-  const int pp = blockIdx.y % p.pairs_per_group;
-  const int h0 = g * p.G + 2 * pp;
-  const bool has1 = (2 * pp + 1) < p.G;
-  const int h1 = h0 + 1;
-
-  const int last_q = min(q0 + kPfTile - 1, len - 1);
-  const int j_hi = last_q / kPfTile;
-  const int j_lo = p.window > 0 ? max(0, q0 - p.window + 1) / kPfTile : 0;
-  const int n_kt = j_hi - j_lo + 1;
 
   if (warp == 8) {
     if (lane == 0) {
       mbar_init(q_full, 1);
-      mbar_init(&k_full[0], 1);
-      mbar_init(&k_full[1], 1);
-      mbar_init(&k_empty[0], 1);
-      mbar_init(&k_empty[1], 1);
+      mbar_init(q_empty, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&k_full[i], 1);
+        mbar_init(&k_empty[i], 1);
+        mbar_init(&s_full[i], 1);
+        mbar_init(&p_full[i], 128);
+        mbar_init(&o_full[i], 1);
+        mbar_init(&o_empty[i], 128);
+      }
       mbar_init(v_full, 1);
       mbar_init(v_empty, 1);
-      mbar_init(&s_full[0], 1);
-      mbar_init(&s_full[1], 1);
-      mbar_init(&p_full[0], 128);
-      mbar_init(&p_full[1], 128);
-      mbar_init(&o_full[0], 1);
-      mbar_init(&o_full[1], 1);
-      *abort_flag = 0;
+      // sampled once, so every thread of the CTA sees the same decision
+      *abort_flag = timed_out_before() ? 1 : 0;
       fence_mbar_init();
     }
     __syncwarp();
@@ -139,8 +172,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
   const uint32_t sbase = smem_u32(smem);
+  // after a recorded timeout elsewhere, do no work (but still free TMEM)
+  const int rounds = *abort_flag ? 0 : (p.num_items + gridDim.x - 1) / gridDim.x;
+
   if (warp >= 8) {
-    setmaxnreg_dec<80>();
+    setmaxnreg_dec<104>();
   }
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -148,28 +184,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(q_full, has1 ? 2 * kPfQBytes : kPfQBytes);
-#pragma unroll
-      for (int c = 0; c < 3; ++c)
-        tma_load_3d(smem + kPfOffQ0 + c * 16384, &tm_q, q_full, c * 64, h0, b0 + q0);
-      if (has1) {
-#pragma unroll
-        for (int c = 0; c < 3; ++c)
-          tma_load_3d(smem + kPfOffQ1 + c * 16384, &tm_q, q_full, c * 64, h1, b0 + q0);
-      }
-      for (int t = 0; t < n_kt; ++t) {
-        const int row = b0 + (j_lo + t) * kPfTile;
-        const int ks = t & 1;
-        if (t >= 2 && !wait_bounded(&k_empty[ks], ((t >> 1) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&k_full[ks], kPfKBytes);
+      int n = 0;   // items loaded
+      int kt = 0;  // key tiles loaded (all items)
+      bool ok = true;
+      for (int r = 0; ok && r < rounds; ++r) {
+        const int item = pf_item_index(r, blockIdx.x, gridDim.x);
+        if (item >= p.num_items) continue;
+        const PfItem it = pf_decode(p, item);
+        if (!it.valid) continue;
+        // Q buffer is free once the previous item's last score MMA completed
+        if (n > 0 && !(ok = wait_bounded(q_empty, (n - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full, it.has1 ? 2 * kPfQBytes : kPfQBytes);
 #pragma unroll
         for (int c = 0; c < 3; ++c)
-          tma_load_3d(smem + kPfOffK + ks * kPfKBytes + c * 16384, &tm_k, &k_full[ks], c * 64, g, row);
-        if (t >= 1 && !wait_bounded(v_empty, (t - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(v_full, kPfVBytes);
+          tma_load_3d(smem + kPfOffQ0 + c * 16384, &tm_q, q_full, c * 64, it.h0, it.b0 + it.q0);
+        if (it.has1) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tma_load_3d(smem + kPfOffV + c * 16384, &tm_v, v_full, c * 64, g, row);
+          for (int c = 0; c < 3; ++c)
+            tma_load_3d(smem + kPfOffQ1 + c * 16384, &tm_q, q_full, c * 64, it.h0 + 1, it.b0 + it.q0);
+        }
+        for (int t = 0; t < it.n_kt; ++t, ++kt) {
+          const int row = it.b0 + (it.j_lo + t) * kPfTile;
+          const int ks = kt & 1;
+          if (kt >= 2 && !(ok = wait_bounded(&k_empty[ks], ((kt >> 1) - 1) & 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&k_full[ks], kPfKBytes);
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            tma_load_3d(smem + kPfOffK + ks * kPfKBytes + c * 16384, &tm_k, &k_full[ks], c * 64, it.g, row);
+          if (kt >= 1 && !(ok = wait_bounded(v_empty, (kt - 1) & 1, abort_flag))) break;
+          mbar_arrive_expect_tx(v_full, kPfVBytes);
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(smem + kPfOffV + c * 16384, &tm_v, v_full, c * 64, it.g, row);
+        }
+        ++n;
       }
     }
   } else if (warp == 9) {
@@ -179,7 +227,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
       const uint32_t tS0 = tbase + 0, tS1 = tbase + 128, tO0 = tbase + 256, tO1 = tbase + 384;
       const uint32_t aQ0 = sbase + kPfOffQ0, aQ1 = sbase + kPfOffQ1;
-      bool ok = wait_bounded(q_full, 0, abort_flag);
       // S_i = Q_i K^T over 192 dims = 12 MMAs of K=16 (3 swizzle boxes x 4 steps of 32 B)
       auto issue_s = [&](uint32_t tS, uint32_t aQ, uint32_t aK) {
 #pragma unroll
@@ -195,73 +242,101 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tO, tP + kk * 8, mnmajor_desc(aV + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
-      if (ok) ok = wait_bounded(&k_full[0], 0, abort_flag);
-      if (ok) {
+      int n = 0;           // items
+      int n1 = 0;          // items with a second head
+      int kt = 0;          // key tiles (all items): K ring and V phases
+      int t0 = 0, t1 = 0;  // score tiles of head 0 / head 1: s_full / p_full phases
+      bool ok = true;
+      for (int r = 0; ok && r < rounds; ++r) {
+        const int item = pf_item_index(r, blockIdx.x, gridDim.x);
+        if (item >= p.num_items) continue;
+        const PfItem it = pf_decode(p, item);
+        if (!it.valid) continue;
+        if (!(ok = wait_bounded(q_full, n & 1, abort_flag))) break;
+        if (!(ok = wait_bounded(&k_full[kt & 1], (kt >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        const uint32_t aK = sbase + kPfOffK;
-        issue_s(tS0, aQ0, aK);
-        umma_commit(&s_full[0]);
-        if (has1) {
-          issue_s(tS1, aQ1, aK);
-          umma_commit(&s_full[1]);
-        }
-        umma_commit(&k_empty[0]);
-      }
-      for (int t = 0; ok && t < n_kt; ++t) {
-        const bool last = (t == n_kt - 1);
-        if (!wait_bounded(v_full, t & 1, abort_flag)) break;
-        if (!wait_bounded(&p_full[0], t & 1, abort_flag)) break;
-        tc_fence_after();
-        issue_pv(tO0, tS0, t > 0);
-        if (last) umma_commit(&o_full[0]);
-        const int kn = (t + 1) & 1;
-        if (!last) {
-          if (!wait_bounded(&k_full[kn], ((t + 1) >> 1) & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_s(tS0, aQ0, sbase + kPfOffK + kn * kPfKBytes);
+        {
+          const uint32_t aK = sbase + kPfOffK + (kt & 1) * kPfKBytes;
+          issue_s(tS0, aQ0, aK);
           umma_commit(&s_full[0]);
-        }
-        if (has1) {
-          if (!wait_bounded(&p_full[1], t & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_pv(tO1, tS1, t > 0);
-          if (last) umma_commit(&o_full[1]);
-        }
-        umma_commit(v_empty);
-        if (!last) {
-          if (has1) {
-            issue_s(tS1, aQ1, sbase + kPfOffK + kn * kPfKBytes);
+          if (it.has1) {
+            issue_s(tS1, aQ1, aK);
             umma_commit(&s_full[1]);
           }
-          umma_commit(&k_empty[kn]);
+          umma_commit(&k_empty[kt & 1]);
+          if (it.n_kt == 1) umma_commit(q_empty);
         }
+        for (int t = 0; t < it.n_kt; ++t, ++kt) {
+          const bool last = (t == it.n_kt - 1);
+          if (!(ok = wait_bounded(v_full, kt & 1, abort_flag))) break;
+          if (!(ok = wait_bounded(&p_full[0], t0 & 1, abort_flag))) break;
+          // O_0 is free once the previous item's epilogue has read it
+          if (t == 0 && n > 0 && !(ok = wait_bounded(&o_empty[0], (n - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(tO0, tS0, t > 0);
+          ++t0;
+          if (last) umma_commit(&o_full[0]);
+          const int kn = kt + 1;
+          if (!last) {
+            if (!(ok = wait_bounded(&k_full[kn & 1], (kn >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_s(tS0, aQ0, sbase + kPfOffK + (kn & 1) * kPfKBytes);
+            umma_commit(&s_full[0]);
+            if (!it.has1 && t + 1 == it.n_kt - 1) umma_commit(q_empty);
+          }
+          if (it.has1) {
+            if (!(ok = wait_bounded(&p_full[1], t1 & 1, abort_flag))) break;
+            if (t == 0 && n1 > 0 && !(ok = wait_bounded(&o_empty[1], (n1 - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_pv(tO1, tS1, t > 0);
+            ++t1;
+            if (last) umma_commit(&o_full[1]);
+          }
+          umma_commit(v_empty);
+          if (!last) {
+            if (it.has1) {
+              issue_s(tS1, aQ1, sbase + kPfOffK + (kn & 1) * kPfKBytes);
+              umma_commit(&s_full[1]);
+              if (t + 1 == it.n_kt - 1) umma_commit(q_empty);
+            }
+            umma_commit(&k_empty[kn & 1]);
+          }
+        }
+        ++n;
+        if (it.has1) ++n1;
       }
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
-    setmaxnreg_inc<208>();
+    setmaxnreg_inc<200>();
     const int i = warp >> 2;  // which head of the pair
-    if (i == 0 || has1) {
-      const int h = i ? h1 : h0;
-      const int r = threadIdx.x & 127;  // TMEM lane == query row within the tile
-      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-      const uint32_t tS = tbase + lane_off + i * 128;
-      const uint32_t tO = tbase + lane_off + 256 + i * 128;
-      const int qpos = q0 + r;
+    const int r = threadIdx.x & 127;  // TMEM lane == query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + lane_off + i * 128;
+    const uint32_t tO = tbase + lane_off + 256 + i * 128;
+    int n = 0;   // items this head slot took part in
+    int tg = 0;  // score tiles this head slot consumed
+    bool ok = true;
+    for (int rr = 0; ok && rr < rounds; ++rr) {
+      const int item = pf_item_index(rr, blockIdx.x, gridDim.x);
+      if (item >= p.num_items) continue;
+      const PfItem it = pf_decode(p, item);
+      if (!it.valid || (i == 1 && !it.has1)) continue;
+      const int h = it.h0 + i;
+      const int qpos = it.q0 + r;
       const float sg2 = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
       float m = sg2;
       float l = p.sinks ? 1.f : 0.f;
-      bool ok = true;
-      for (int t = 0; t < n_kt; ++t) {
-        const int kpos0 = (j_lo + t) * kPfTile;
-        if (!wait_bounded(&s_full[i], t & 1, abort_flag)) { ok = false; break; }
+      for (int t = 0; t < it.n_kt; ++t, ++tg) {
+        const int kpos0 = (it.j_lo + t) * kPfTile;
+        if (!(ok = wait_bounded(&s_full[i], tg & 1, abort_flag))) break;
         tc_fence_after();
         float s[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32f(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
         tmem_wait_ld();
-        const bool full_tile = (kpos0 + kPfTile - 1 <= q0) &&
-                               (p.window == 0 || (q0 + kPfTile - 1) - kpos0 <= p.window - 1);
+        const bool full_tile = (kpos0 + kPfTile - 1 <= it.q0) &&
+                               (p.window == 0 || (it.q0 + kPfTile - 1) - kpos0 <= p.window - 1);
         // Row max of the raw scores (the scale is positive, so it commutes with
         // max), as 8 independent chains to keep the dependency depth short.
         float mx8[8];
@@ -311,8 +386,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
         const float2 a = add2(a01, a23);
-        const float rs = a.x + a.y;
-        l += rs;
+        l += a.x + a.y;
         // O of the previous tile is complete here: S_i(t) was committed after PV_i(t-1).
         if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
@@ -320,9 +394,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             uint32_t o[32];
             tmem_ld32(tO + c * 32, o);
             tmem_wait_ld();
-            const float a = rescale_o ? alpha : 1.f;
+            const float a_ = rescale_o ? alpha : 1.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a_);
             tmem_st32(tO + c * 32, o);
           }
         }
@@ -330,40 +404,62 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_before();
         mbar_arrive(&p_full[i]);
       }
-      // ---------------- epilogue: O / l -> out, lse
-      if (ok && wait_bounded(&o_full[i], 0, abort_flag)) {
-        tc_fence_after();
-        const bool valid = qpos < len;
-        const int tok = b0 + qpos;
+      if (!ok) break;
+      // ---------------- epilogue: O / l -> out, lse.  O is read out of TMEM
+      // first and released, so the next item's P.V can start at once.
+      if (!(ok = wait_bounded(&o_full[i], n & 1, abort_flag))) break;
+      tc_fence_after();
+      float o[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32f(tO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&o_empty[i]);
+      ++n;
+      if (qpos < it.len) {
+        const int tok = it.b0 + qpos;
         const float f = (l > 0.f) ? p.v_scale / l : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          if (valid) {
-            const size_t ob = ((size_t)tok * p.Hq + h) * 128 + c * 32;
-            if (p.out_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob);
+        const size_t ob = ((size_t)tok * p.Hq + h) * 128;
+        if (p.out_f32) {
+          float* dst = reinterpret_cast<float*>(p.out) + ob;
+          if (p.out_v8) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(o[4 * e]) * f, __uint_as_float(o[4 * e + 1]) * f,
-                                     __uint_as_float(o[4 * e + 2]) * f, __uint_as_float(o[4 * e + 3]) * f);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob);
+            for (int e = 0; e < 16; ++e)
+              st_global_v8(dst + 8 * e, __float_as_uint(o[8 * e] * f), __float_as_uint(o[8 * e + 1] * f),
+                           __float_as_uint(o[8 * e + 2] * f), __float_as_uint(o[8 * e + 3] * f),
+                           __float_as_uint(o[8 * e + 4] * f), __float_as_uint(o[8 * e + 5] * f),
+                           __float_as_uint(o[8 * e + 6] * f), __float_as_uint(o[8 * e + 7] * f));
+          } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                uint4 u;
-                u.x = pack_bf16(__uint_as_float(o[8 * e + 0]) * f, __uint_as_float(o[8 * e + 1]) * f);
-                u.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * f, __uint_as_float(o[8 * e + 3]) * f);
-                u.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * f, __uint_as_float(o[8 * e + 5]) * f);
-                u.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * f, __uint_as_float(o[8 * e + 7]) * f);
-                dst[e] = u;
-              }
-            }
+            for (int e = 0; e < 32; ++e)
+              reinterpret_cast<float4*>(dst)[e] =
+                  make_float4(o[4 * e] * f, o[4 * e + 1] * f, o[4 * e + 2] * f, o[4 * e + 3] * f);
+          }
+        } else if (p.out_v8) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ob;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            st_global_v8(dst + 16 * e, pack_bf16(o[16 * e + 0] * f, o[16 * e + 1] * f),
+                         pack_bf16(o[16 * e + 2] * f, o[16 * e + 3] * f),
+                         pack_bf16(o[16 * e + 4] * f, o[16 * e + 5] * f),
+                         pack_bf16(o[16 * e + 6] * f, o[16 * e + 7] * f),
+                         pack_bf16(o[16 * e + 8] * f, o[16 * e + 9] * f),
+                         pack_bf16(o[16 * e + 10] * f, o[16 * e + 11] * f),
+                         pack_bf16(o[16 * e + 12] * f, o[16 * e + 13] * f),
+                         pack_bf16(o[16 * e + 14] * f, o[16 * e + 15] * f));
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            uint4 u;
+            u.x = pack_bf16(o[8 * e + 0] * f, o[8 * e + 1] * f);
+            u.y = pack_bf16(o[8 * e + 2] * f, o[8 * e + 3] * f);
+            u.z = pack_bf16(o[8 * e + 4] * f, o[8 * e + 5] * f);
+            u.w = pack_bf16(o[8 * e + 6] * f, o[8 * e + 7] * f);
+            dst[e] = u;
           }
         }
-        if (valid && p.lse)
+        if (p.lse)
           p.lse[(size_t)h * p.total + tok] = (l > 0.f) ? (m * 0.6931471805599453f + logf(l)) : -INFINITY;
       }
     }

@@ -161,3 +161,19 @@ def test_full_size_varlen_stack():
     sinks = W.stack_sinks(len(W.STACK_WINDOWS), seed=0)
     for layer, window in enumerate(W.STACK_WINDOWS):
         full_size_check(lengths, window, seed=100 + layer, per_seq_random=4, sinks=sinks[layer])
+
+
+@pytest.mark.parametrize("odt", [torch.bfloat16, torch.float32])
+def test_output_only_16_byte_aligned(odt):
+    """An output pointer aligned to 16 but not 32 bytes takes the 16-byte store path."""
+    x = W.prefill_inputs([300], hq=4, hkv=1, seed=17)
+    n = 300 * 4 * 128
+    flat = torch.empty(n + 16, dtype=odt, device="cuda")
+    shift = 16 // flat.element_size()
+    out = flat[shift:shift + n].view(300, 4, 128)
+    assert out.data_ptr() % 32 == 16
+    mimo.mimo_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.sinks.cuda(), 129,
+                           x.cu_seqlens.cuda(), 300, out=out)
+    mimo.mimo_attn_device_status()
+    ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, 129, x.cu_seqlens)
+    P.check(out, ro, what="16-byte aligned out")
