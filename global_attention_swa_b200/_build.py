@@ -11,7 +11,8 @@ SRC = os.path.join(PKG, "csrc", "mimo_attn.cu")
 LIB = os.path.join(PKG, "libmimo_attn.so")
 DEPS = [
     os.path.join(PKG, "csrc", f)
-    for f in ("mimo_attn.cu", "common.cuh", "decode_kernel.cuh", "prefill_kernel.cuh")
+    for f in ("mimo_attn.cu", "common.cuh", "decode_kernel.cuh", "prefill_kernel.cuh",
+              "prefill_swa_kernel.cuh")
 ] + [os.path.join(ROOT, "include", "mimo_attn.h")]
 
 NVCC_FLAGS = [

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "decode_kernel.cuh"
 #include "prefill_kernel.cuh"
+#include "prefill_swa_kernel.cuh"
 
 namespace {
 
@@ -125,6 +126,11 @@ mimo_status_t ensure_attributes() {
                                             mimo::kPfSmemBytes),
                        "prefill smem attribute")))
     return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::prefill_swa_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kSwSmemBytes),
+                       "sliding-window prefill smem attribute")))
+    return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kDecSmemBytes),
@@ -218,6 +224,58 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
   if (num_seqs > 65535) return fail(MIMO_ERR_UNSUPPORTED, "num_seqs > 65535");
   const int Hq = dims->num_heads_q, Hkv = dims->num_heads_kv, G = Hq / Hkv;
   if ((st = ensure_attributes())) return st;
+
+  // Sliding window with the key/value group packed into one 128-row tile:
+  // 128 / G queries x G heads per block, one score tile of N keys per block.
+  const int QB = (G >= 8 && 128 % G == 0) ? 128 / G : 0;
+  const int Nsw = QB ? ((window + QB - 1 + 15) / 16) * 16 : 0;
+  if (window > 0 && QB > 0 && Nsw <= mimo::kSwNMax) {
+    CUtensorMap tq, tk, tv;
+    {
+      const uint64_t d[3] = {192, (uint64_t)Hq, (uint64_t)total_tokens};
+      const uint64_t s[2] = {192 * 2, (uint64_t)Hq * 192 * 2};
+      const uint32_t b[3] = {64, (uint32_t)G, (uint32_t)QB};
+      if ((st = make_map(&tq, q, 3, d, s, b))) return st;
+    }
+    {
+      const uint64_t d[3] = {192, (uint64_t)Hkv, (uint64_t)total_tokens};
+      const uint64_t s[2] = {192 * 2, (uint64_t)Hkv * 192 * 2};
+      const uint32_t b[3] = {64, 1, (uint32_t)Nsw};
+      if ((st = make_map(&tk, k, 3, d, s, b))) return st;
+    }
+    {
+      const uint64_t d[3] = {128, (uint64_t)Hkv, (uint64_t)total_tokens};
+      const uint64_t s[2] = {128 * 2, (uint64_t)Hkv * 128 * 2};
+      const uint32_t b[3] = {64, 1, (uint32_t)Nsw};
+      if ((st = make_map(&tv, v, 3, d, s, b))) return st;
+    }
+    mimo::SwaParams sp;
+    sp.cu_seqlens = cu_seqlens;
+    sp.sinks = sinks;
+    sp.out = out;
+    sp.lse = lse;
+    sp.total = total_tokens;
+    sp.Hq = Hq;
+    sp.Hkv = Hkv;
+    sp.G = G;
+    sp.QB = QB;
+    sp.N = Nsw;
+    sp.window = window;
+    sp.num_seqs = num_seqs;
+    sp.num_qblocks = (max_seqlen + QB - 1) / QB;
+    const long items = (long)sp.num_qblocks * Hkv * num_seqs;
+    if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
+    sp.num_items = (int)items;
+    sp.scale_log2 = scale_log2_of(dims);
+    sp.v_scale = v_scale_of(dims);
+    sp.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+    sp.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    const int grid = (int)std::min<long>(items, sm_count());
+    mimo::prefill_swa_kernel<<<grid, mimo::kSwThreads, mimo::kSwSmemBytes, (cudaStream_t)stream>>>(
+        tq, tk, tv, sp);
+    if ((st = cuda_check(cudaGetLastError(), "sliding-window prefill launch"))) return st;
+    return ok();
+  }
 
   CUtensorMap tq, tk, tv;
   {

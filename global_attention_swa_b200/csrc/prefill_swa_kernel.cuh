@@ -1,0 +1,371 @@
+// Sliding-window prefill with the whole key/value group packed into the MMA
+// rows (tcgen05).
+//
+// MiMo-V2-Flash model doc, "Key features" (sliding-window layers with a small
+// window, learnable attention sink) and MiMoV2FlashConfig (64 query heads
+// over 4 key/value heads, head_dim 192 / v_head_dim 128, sliding_window 129).
+//
+// A block is QB = 128 / G consecutive queries of one sequence times the G
+// query heads of one key/value head g: 128 rows, row = query * G + head (the
+// [token][head][dim] layout makes these rows one TMA box).  All G heads read
+// the same keys, so one score tile covers the block: its key window is the
+// N = roundup16(W + QB - 1) keys [q0 + QB - N, q0 + QB), of which each row
+// sees at most W (~90 % useful at W = 129, QB = 8, N = 144).  With the whole
+// window in one tile there is no online rescaling: max, exponentials and the
+// sink's share are exact for the row.
+//
+//   warp 8      TMA producer: Q double-buffered (2 x 48 KB, from DRAM, one
+//               block ahead), K (N x 384 B) and V (N x 256 B) single.
+//   warp 9      MMA issuer: S(n) = Q K^T into one of two TMEM score buffers,
+//               then O = P(n-1) V for the previous block (software pipelined).
+//   warps 0-3   softmax: one row per thread, two passes over the TMEM row
+//               (max, then exponentials), P written back as bf16.
+//   warps 4-7   epilogue: O / l -> bf16/fp32 rows, lse.
+//   warps 10-11 idle (complete the third warpgroup)
+//
+// TMEM: S_0 [0, 192), S_1 [192, 384), O [384, 512).
+#pragma once
+
+#include "common.cuh"
+
+namespace mimo {
+
+constexpr int kSwThreads = 384;
+constexpr int kSwNMax = 192;
+constexpr int kSwQBytes = 3 * 16384;                   // [128 rows][192 dims] as 3 boxes
+constexpr int kSwKBox = kSwNMax * 128;                 // [N rows][64 dims], 1024-aligned
+constexpr int kSwOffQ = 0;                             // 2 buffers
+constexpr int kSwOffK = 2 * kSwQBytes;                 // 98304: 3 boxes
+constexpr int kSwOffV = kSwOffK + 3 * kSwKBox;         // 172032: 2 boxes
+constexpr int kSwOffML = kSwOffV + 2 * kSwKBox;        // 221184: [2][128] float2
+constexpr int kSwOffBar = kSwOffML + 2 * 128 * 8;      // 223232
+constexpr int kSwSmemBytes = kSwOffBar + 256 + 1024;
+
+struct SwaParams {
+  const int32_t* cu_seqlens;
+  const float* sinks;
+  void* out;
+  float* lse;
+  int total, Hq, Hkv, G, QB, N, window;
+  int num_seqs, num_qblocks, num_items;
+  float scale_log2, v_scale;
+  int out_f32, out_v8;
+};
+
+struct SwItem {
+  int b0, len, q0, g;
+  bool valid;
+};
+
+__device__ __forceinline__ SwItem sw_decode(const SwaParams& p, int item) {
+  SwItem it;
+  const int per_qb = p.Hkv * p.num_seqs;
+  const int qb = item / per_qb;
+  const int rem = item % per_qb;
+  const int seq = rem / p.Hkv;
+  it.g = rem % p.Hkv;
+  it.b0 = p.cu_seqlens[seq];
+  it.len = p.cu_seqlens[seq + 1] - it.b0;
+  it.q0 = qb * p.QB;
+  it.valid = it.q0 < it.len;
+  return it;
+}
+
+// First valid item at or after round r of this CTA (round-robin); -1 if none.
+__device__ __forceinline__ int sw_next(const SwaParams& p, int r, int rounds, SwItem& it) {
+  for (; r < rounds; ++r) {
+    const int item = r * gridDim.x + blockIdx.x;
+    if (item >= p.num_items) return -1;
+    it = sw_decode(p, item);
+    if (it.valid) return r;
+  }
+  return -1;
+}
+
+__global__ void __launch_bounds__(kSwThreads, 1)
+    prefill_swa_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const SwaParams p) {
+  extern __shared__ __align__(1024) uint8_t ssmem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(ssmem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSwOffBar);
+  uint64_t* q_full = bars + 0;    // [2]
+  uint64_t* q_empty = bars + 2;   // [2]
+  uint64_t* k_full = bars + 4;
+  uint64_t* k_empty = bars + 5;
+  uint64_t* v_full = bars + 6;
+  uint64_t* v_empty = bars + 7;
+  uint64_t* s_full = bars + 8;    // [2]
+  uint64_t* p_full = bars + 10;   // [2]
+  uint64_t* o_full = bars + 12;
+  uint64_t* o_empty = bars + 13;
+  uint64_t* ml_full = bars + 14;  // [2]
+  uint64_t* ml_empty = bars + 16; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
+  float2* ml = reinterpret_cast<float2*>(smem + kSwOffML);  // [2][128] (m, l) per row
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 8) {
+    if (lane == 0) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&q_full[i], 1);
+        mbar_init(&q_empty[i], 1);
+        mbar_init(&s_full[i], 1);
+        mbar_init(&p_full[i], 128);
+        mbar_init(&ml_full[i], 128);
+        mbar_init(&ml_empty[i], 128);
+      }
+      mbar_init(k_full, 1);
+      mbar_init(k_empty, 1);
+      mbar_init(v_full, 1);
+      mbar_init(v_empty, 1);
+      mbar_init(o_full, 1);
+      mbar_init(o_empty, 128);
+      *abort_flag = timed_out_before() ? 1 : 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t sbase = smem_u32(smem);
+  const int rounds = *abort_flag ? 0 : (p.num_items + gridDim.x - 1) / gridDim.x;
+  const int N = p.N;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      auto load_q = [&](const SwItem& it, int b) {
+        mbar_arrive_expect_tx(&q_full[b], kSwQBytes);
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          tma_load_3d(smem + kSwOffQ + b * kSwQBytes + c * 16384, &tm_q, &q_full[b], c * 64,
+                      it.g * p.G, it.b0 + it.q0);
+      };
+      SwItem cur, nxt;
+      int r = sw_next(p, 0, rounds, cur);
+      if (r >= 0) load_q(cur, 0);
+      bool ok = true;
+      for (int n = 0; ok && r >= 0; ++n) {
+        const int k0 = cur.q0 + p.QB - N;  // may be negative: zero-filled or masked
+        if (n >= 1 && !(ok = wait_bounded(k_empty, (n - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(k_full, 3 * N * 128);
+#pragma unroll
+        for (int c = 0; c < 3; ++c)
+          tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
+        // next block's Q, one block ahead (its buffer was freed by S(n-1))
+        const int rn = sw_next(p, r + 1, rounds, nxt);
+        if (rn >= 0) {
+          const int bn = (n + 1) & 1;
+          if (n + 1 >= 2 && !(ok = wait_bounded(&q_empty[bn], (((n + 1) >> 1) - 1) & 1, abort_flag))) break;
+          load_q(nxt, bn);
+        }
+        if (n >= 1 && !(ok = wait_bounded(v_empty, (n - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(v_full, 2 * N * 128);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(smem + kSwOffV + c * kSwKBox, &tm_v, v_full, c * 64, cur.g, cur.b0 + k0);
+        cur = nxt;
+        r = rn;
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, N, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t tO = tbase + 384;
+      bool ok = true;
+      // O = P(m) V over N keys: N/16 MMAs (P: 8 TMEM columns each; V: 16 rows = 2 KB)
+      auto do_pv = [&](int m) {
+        const int bm = m & 1;
+        if (!(ok = wait_bounded(&p_full[bm], (m >> 1) & 1, abort_flag))) return;
+        if (!(ok = wait_bounded(v_full, m & 1, abort_flag))) return;
+        if (m >= 1 && !(ok = wait_bounded(o_empty, (m - 1) & 1, abort_flag))) return;
+        tc_fence_after();
+        const uint32_t tP = tbase + bm * kSwNMax;
+        const uint32_t aV = sbase + kSwOffV;
+        for (int kk = 0; kk < N / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, smem_desc_sw128(aV + kk * 2048, kSwKBox, 1024), idesc_o,
+                  kk > 0 ? 1u : 0u);
+        umma_commit(o_full);
+        umma_commit(v_empty);
+      };
+      SwItem it;
+      int n = 0;
+      for (int r = sw_next(p, 0, rounds, it); ok && r >= 0; r = sw_next(p, r + 1, rounds, it), ++n) {
+        const int b = n & 1;
+        if (!(ok = wait_bounded(&q_full[b], (n >> 1) & 1, abort_flag))) break;
+        if (!(ok = wait_bounded(k_full, n & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t aQ = sbase + kSwOffQ + b * kSwQBytes;
+        const uint32_t aK = sbase + kSwOffK;
+        const uint32_t tS = tbase + b * kSwNMax;
+#pragma unroll
+        for (int kk = 0; kk < 12; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          umma_ss(tS, smem_desc_sw128(aQ + (kk >> 2) * 16384 + off, 16, 1024),
+                  smem_desc_sw128(aK + (kk >> 2) * kSwKBox + off, 16, 1024), idesc_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[b]);
+        umma_commit(k_empty);
+        umma_commit(&q_empty[b]);
+        if (n >= 1) do_pv(n - 1);
+      }
+      if (ok && n >= 1) do_pv(n - 1);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    const int r = threadIdx.x;  // TMEM lane = row = query * G + head
+    const int a = r / p.G, hh = r % p.G;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    SwItem it;
+    int n = 0;
+    bool ok = true;
+    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it), ++n) {
+      const int b = n & 1;
+      const int hg = it.g * p.G + hh;
+      const int qpos = it.q0 + a;
+      const int k0 = it.q0 + p.QB - N;
+      const int c_hi = qpos - k0;                              // keys <= qpos
+      const int c_lo = max(qpos - p.window + 1, 0) - k0;       // keys in window, >= 0
+      const float sg2 = p.sinks ? p.sinks[hg] * 1.4426950408889634f : -INFINITY;
+      if (!(ok = wait_bounded(&s_full[b], (n >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t tS = tbase + lane_off + b * kSwNMax;
+      // pass 1: row max over the visible columns
+      float mx = -INFINITY;
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tS + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = c0 + e;
+          if (c >= c_lo && c <= c_hi) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
+      }
+      float m = fmaxf(sg2, mx * p.scale_log2);
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same columns
+      float l0 = 0.f, l1 = 0.f;
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t v[16], pk[8];
+        tmem_ld16(tS + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = c0 + 2 * e;
+          const float x0 = fmaf(__uint_as_float(v[2 * e]), p.scale_log2, neg_m);
+          const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, neg_m);
+          const float p0 = (c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f;
+          const float p1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f;
+          l0 += p0;
+          l1 += p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st8(tS + c0 / 2, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+      float l = l0 + l1;
+      if (p.sinks && m != -INFINITY) l += ex2(sg2 - m);
+      if (n >= 2 && !(ok = wait_bounded(&ml_empty[b], ((n >> 1) - 1) & 1, abort_flag))) break;
+      ml[b * 128 + r] = make_float2(m, l);
+      mbar_arrive(&ml_full[b]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ epilogue
+    const int r = threadIdx.x - 128;
+    const int a = r / p.G, hh = r % p.G;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tO = tbase + lane_off + 384;
+    SwItem it;
+    int n = 0;
+    bool ok = true;
+    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it), ++n) {
+      const int b = n & 1;
+      if (!(ok = wait_bounded(o_full, n & 1, abort_flag))) break;
+      tc_fence_after();
+      float o[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32f(tO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(o_empty);
+      if (!(ok = wait_bounded(&ml_full[b], (n >> 1) & 1, abort_flag))) break;
+      const float2 mlv = ml[b * 128 + r];
+      mbar_arrive(&ml_empty[b]);
+      const int qpos = it.q0 + a;
+      if (qpos < it.len) {
+        const int tok = it.b0 + qpos;
+        const int hg = it.g * p.G + hh;
+        const float l = mlv.y;
+        const float f = (l > 0.f) ? p.v_scale / l : 0.f;
+        const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
+        if (p.out_f32) {
+          float* dst = reinterpret_cast<float*>(p.out) + ob;
+          if (p.out_v8) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              st_global_v8(dst + 8 * e, __float_as_uint(o[8 * e] * f), __float_as_uint(o[8 * e + 1] * f),
+                           __float_as_uint(o[8 * e + 2] * f), __float_as_uint(o[8 * e + 3] * f),
+                           __float_as_uint(o[8 * e + 4] * f), __float_as_uint(o[8 * e + 5] * f),
+                           __float_as_uint(o[8 * e + 6] * f), __float_as_uint(o[8 * e + 7] * f));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              reinterpret_cast<float4*>(dst)[e] =
+                  make_float4(o[4 * e] * f, o[4 * e + 1] * f, o[4 * e + 2] * f, o[4 * e + 3] * f);
+          }
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ob;
+          if (p.out_v8) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              st_global_v8(dst + 16 * e, pack_bf16(o[16 * e + 0] * f, o[16 * e + 1] * f),
+                           pack_bf16(o[16 * e + 2] * f, o[16 * e + 3] * f),
+                           pack_bf16(o[16 * e + 4] * f, o[16 * e + 5] * f),
+                           pack_bf16(o[16 * e + 6] * f, o[16 * e + 7] * f),
+                           pack_bf16(o[16 * e + 8] * f, o[16 * e + 9] * f),
+                           pack_bf16(o[16 * e + 10] * f, o[16 * e + 11] * f),
+                           pack_bf16(o[16 * e + 12] * f, o[16 * e + 13] * f),
+                           pack_bf16(o[16 * e + 14] * f, o[16 * e + 15] * f));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              uint4 u;
+              u.x = pack_bf16(o[8 * e + 0] * f, o[8 * e + 1] * f);
+              u.y = pack_bf16(o[8 * e + 2] * f, o[8 * e + 3] * f);
+              u.z = pack_bf16(o[8 * e + 4] * f, o[8 * e + 5] * f);
+              u.w = pack_bf16(o[8 * e + 6] * f, o[8 * e + 7] * f);
+              reinterpret_cast<uint4*>(dst)[e] = u;
+            }
+          }
+        }
+        if (p.lse)
+          p.lse[(size_t)hg * p.total + tok] =
+              (l > 0.f) ? (mlv.x * 0.6931471805599453f + logf(l)) : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace mimo

@@ -177,3 +177,42 @@ def test_output_only_16_byte_aligned(odt):
     mimo.mimo_attn_device_status()
     ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, 129, x.cu_seqlens)
     P.check(out, ro, what="16-byte aligned out")
+
+
+# ----------------------------------------------------------------------------
+# sliding window with the key/value group packed into the MMA rows
+# (G = Hq/Hkv in {8, 16, 32}; N = roundup16(W + 128/G - 1) <= 192, else the
+# general kernel takes the call)
+
+
+@pytest.mark.parametrize("hq,hkv", [(16, 1), (16, 2), (64, 2)])
+@pytest.mark.parametrize("window", [1, 2, 8, 128, 129, 130, 177, 185, 186])
+def test_packed_window_lengths(hq, hkv, window):
+    for T in (1, 2, 7, 8, 9, 127, 129, 300, 1000):
+        sinks = (T + window) % 3 != 0
+        x = W.prefill_inputs([T], hq=hq, hkv=hkv, seed=T * 31 + window + hq, sinks=sinks)
+        out, lse = run_gpu(x, window, torch.float32 if T % 2 else torch.bfloat16)
+        ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+        P.check(out, ro, lse, rl, what=f"packed Hq={hq} Hkv={hkv} T={T} W={window}")
+
+
+@pytest.mark.parametrize("window", [129, 5])
+def test_packed_window_varlen(window):
+    lengths = [0, 1, 300, 0, 129, 1000, 5, 128, 7]
+    x = W.prefill_inputs(lengths, hq=16, hkv=1, seed=88 + window)
+    out, lse = run_gpu(x, window, torch.bfloat16)
+    ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+    P.check(out, ro, lse, rl, what=f"packed varlen W={window}")
+
+
+def test_packed_window_16_byte_aligned_output():
+    x = W.prefill_inputs([300], hq=16, hkv=1, seed=19)
+    n = 300 * 16 * 128
+    flat = torch.empty(n + 8, dtype=torch.bfloat16, device="cuda")
+    out = flat[8:8 + n].view(300, 16, 128)
+    assert out.data_ptr() % 32 == 16
+    mimo.mimo_attn_prefill(x.q.cuda(), x.k.cuda(), x.v.cuda(), x.sinks.cuda(), 129,
+                           x.cu_seqlens.cuda(), 300, out=out)
+    mimo.mimo_attn_device_status()
+    ro, _ = oracle.prefill(x.q, x.k, x.v, x.sinks, 129, x.cu_seqlens)
+    P.check(out, ro, what="packed, 16-byte aligned out")
