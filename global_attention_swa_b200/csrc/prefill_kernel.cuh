@@ -332,9 +332,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!(ok = wait_bounded(&s_full[i], tg & 1, abort_flag))) break;
         tc_fence_after();
         float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32f(tS + c * 32, *reinterpret_cast<float(*)[32]>(&s[c * 32]));
-        tmem_wait_ld();
+        tmem_load128_sync(tS, s);
         const bool full_tile = (kpos0 + kPfTile - 1 <= it.q0) &&
                                (p.window == 0 || (it.q0 + kPfTile - 1) - kpos0 <= p.window - 1);
         // Row max of the raw scores (the scale is positive, so it commutes with
@@ -392,8 +390,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_wait_ld();
+            tmem_load32_sync(tO + c * 32, o);
             const float a_ = rescale_o ? alpha : 1.f;
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a_);
@@ -410,9 +407,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!(ok = wait_bounded(&o_full[i], n & 1, abort_flag))) break;
       tc_fence_after();
       float o[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32f(tO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
-      tmem_wait_ld();
+      tmem_load128_sync(tO, o);
       tc_fence_before();
       mbar_arrive(&o_empty[i]);
       ++n;

@@ -246,8 +246,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       float mx = -INFINITY;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16];
-        tmem_ld16(tS + c0, v);
-        tmem_wait_ld();
+        tmem_load16_sync(tS + c0, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = c0 + e;
@@ -260,8 +259,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       float l0 = 0.f, l1 = 0.f;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16], pk[8];
-        tmem_ld16(tS + c0, v);
-        tmem_wait_ld();
+        tmem_load16_sync(tS + c0, v);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int c = c0 + 2 * e;
@@ -298,9 +296,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       if (!(ok = wait_bounded(o_full, n & 1, abort_flag))) break;
       tc_fence_after();
       float o[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32f(tO + c * 32, *reinterpret_cast<float(*)[32]>(&o[c * 32]));
-      tmem_wait_ld();
+      tmem_load128_sync(tO, o);
       tc_fence_before();
       mbar_arrive(o_empty);
       if (!(ok = wait_bounded(&ml_full[b], (n >> 1) & 1, abort_flag))) break;
