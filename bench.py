@@ -478,6 +478,10 @@ def run_case(args):
     else:
         lengths = W.decode_b64_lengths(0)
         window, cap = (0, W.DECODE_GA_CAPACITY) if args.case == "decode_global" else (SWA, SWA)
+        if args.case == "decode_global" and args.decode_cap:
+            # smaller caches (for profiler captures): lengths ~U[1024, cap]
+            cap = args.decode_cap
+            lengths = W.lengths_uniform(0, 64, 1024, cap)
         d = W.decode_inputs(lengths, cap, window, seed=3, device=dev)
         fn = lambda: mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks)  # noqa: E731
         work = decode_work(lengths, window, cap)
@@ -515,6 +519,8 @@ def main():
                                        "decode_ring"], default="step",
                     help="run one kernel alone (profiling); 'step' is the benchmark")
     ap.add_argument("--seq-len", type=int, default=T_PREFILL, help="prefill length for --case")
+    ap.add_argument("--decode-cap", type=int, default=0,
+                    help="decode_global --case with caches of this capacity (0: 262144)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
