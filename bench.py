@@ -262,7 +262,16 @@ def run_ours(args, rank, world, peaks, peak_kind):
                 "traffic": None}
     tr = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tr):
-        roofline["traffic"] = json.load(open(tr)).get("prefill_global_T32768")
+        import hashlib
+
+        rec = json.load(open(tr))
+        h = hashlib.sha256()
+        for f in rec.get("source_files", []):
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+        # counters taken on another revision of the kernel do not describe this one
+        if h.hexdigest() == rec.get("source_sha256"):
+            roofline["traffic"] = rec.get("prefill_global_T32768")
 
     # --- e2e through the public API with pinned host buffers
     e2e = None
