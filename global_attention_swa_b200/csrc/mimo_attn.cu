@@ -228,7 +228,7 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
   // Sliding window with the key/value group packed into one 128-row tile:
   // 128 / G queries x G heads per block, one score tile of N keys per block.
   const int QB = (G >= 8 && 128 % G == 0) ? 128 / G : 0;
-  const int Nsw = QB ? ((window + QB - 1 + 15) / 16) * 16 : 0;
+  const int Nsw = QB ? ((window + 2 * QB - 1 + 15) / 16) * 16 : 0;  // window of a block pair
   if (window > 0 && QB > 0 && Nsw <= mimo::kSwNMax) {
     CUtensorMap tq, tk, tv;
     {
@@ -262,8 +262,8 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
     sp.N = Nsw;
     sp.window = window;
     sp.num_seqs = num_seqs;
-    sp.num_qblocks = (max_seqlen + QB - 1) / QB;
-    const long items = (long)sp.num_qblocks * Hkv * num_seqs;
+    sp.num_pairs = (max_seqlen + 2 * QB - 1) / (2 * QB);
+    const long items = (long)sp.num_pairs * Hkv * num_seqs;
     if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
     sp.num_items = (int)items;
     sp.scale_log2 = scale_log2_of(dims);

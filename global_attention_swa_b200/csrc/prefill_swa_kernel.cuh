@@ -8,14 +8,15 @@
 // A block is QB = 128 / G consecutive queries of one sequence times the G
 // query heads of one key/value head g: 128 rows, row = query * G + head (the
 // [token][head][dim] layout makes these rows one TMA box).  All G heads read
-// the same keys, so one score tile covers the block: its key window is the
-// N = roundup16(W + QB - 1) keys [q0 + QB - N, q0 + QB), of which each row
-// sees at most W (~90 % useful at W = 129, QB = 8, N = 144).  With the whole
-// window in one tile there is no online rescaling: max, exponentials and the
-// sink's share are exact for the row.
+// the same keys, so one score tile covers the block.  Blocks go in pairs (2 QB
+// queries): both blocks of a pair share one key window, the
+// N = roundup16(W + 2 QB - 1) keys [q0 + 2 QB - N, q0 + 2 QB), loaded once,
+// of which each row sees at most W (~90 % useful at W = 129, QB = 8, N = 144).
+// With the whole window in one tile there is no online rescaling: max,
+// exponentials and the sink's share are exact for the row.
 //
 //   warp 8      TMA producer: Q double-buffered (2 x 48 KB, from DRAM, one
-//               block ahead), K (N x 384 B) and V (N x 256 B) single.
+//               block ahead), K (N x 384 B) and V (N x 256 B) once per pair.
 //   warp 9      MMA issuer: S(n) = Q K^T into one of two TMEM score buffers,
 //               then O = P(n-1) V for the previous block (software pipelined).
 //   warps 0-3   softmax: one row per thread, two passes over the TMEM row
@@ -47,13 +48,14 @@ struct SwaParams {
   void* out;
   float* lse;
   int total, Hq, Hkv, G, QB, N, window;
-  int num_seqs, num_qblocks, num_items;
+  int num_seqs, num_pairs, num_items;   // items = pairs of blocks
   float scale_log2, v_scale;
   int out_f32, out_v8;
 };
 
+// A work item is a pair of blocks: queries [q0, q0 + 2 QB) of one sequence.
 struct SwItem {
-  int b0, len, q0, g;
+  int b0, len, q0, g, nblk;  // nblk: 1 or 2 valid blocks
   bool valid;
 };
 
@@ -66,8 +68,9 @@ __device__ __forceinline__ SwItem sw_decode(const SwaParams& p, int item) {
   it.g = rem % p.Hkv;
   it.b0 = p.cu_seqlens[seq];
   it.len = p.cu_seqlens[seq + 1] - it.b0;
-  it.q0 = qb * p.QB;
+  it.q0 = qb * 2 * p.QB;
   it.valid = it.q0 < it.len;
+  it.nblk = (it.q0 + p.QB < it.len) ? 2 : 1;
   return it;
 }
 
@@ -143,36 +146,51 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      auto load_q = [&](const SwItem& it, int b) {
+      auto load_q = [&](const SwItem& it, int blk, int b) {
         mbar_arrive_expect_tx(&q_full[b], kSwQBytes);
 #pragma unroll
         for (int c = 0; c < 3; ++c)
           tma_load_3d(smem + kSwOffQ + b * kSwQBytes + c * 16384, &tm_q, &q_full[b], c * 64,
-                      it.g * p.G, it.b0 + it.q0);
+                      it.g * p.G, it.b0 + it.q0 + blk * p.QB);
       };
+      // Blocks are numbered n = 0, 1, ... over this CTA's pairs; block n uses Q
+      // buffer n & 1.  The pair's K/V window is loaded at its first block.
       SwItem cur, nxt;
       int r = sw_next(p, 0, rounds, cur);
-      if (r >= 0) load_q(cur, 0);
+      if (r >= 0) load_q(cur, 0, 0);
       bool ok = true;
-      for (int n = 0; ok && r >= 0; ++n) {
-        const int k0 = cur.q0 + p.QB - N;  // may be negative: zero-filled or masked
-        if (n >= 1 && !(ok = wait_bounded(k_empty, (n - 1) & 1, abort_flag))) break;
-        mbar_arrive_expect_tx(k_full, 3 * N * 128);
+      int n = 0, kp = 0;
+      while (ok && r >= 0) {
+        const int k0 = cur.q0 + 2 * p.QB - N;  // may be negative: zero-filled or masked
+        int rn = -1;
+        for (int blk = 0; ok && blk < cur.nblk; ++blk, ++n) {
+          if (blk == 0) {
+            if (kp >= 1 && !(ok = wait_bounded(k_empty, (kp - 1) & 1, abort_flag))) break;
+            mbar_arrive_expect_tx(k_full, 3 * N * 128);
 #pragma unroll
-        for (int c = 0; c < 3; ++c)
-          tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
-        // next block's Q, one block ahead (its buffer was freed by S(n-1))
-        const int rn = sw_next(p, r + 1, rounds, nxt);
-        if (rn >= 0) {
+            for (int c = 0; c < 3; ++c)
+              tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
+          }
+          // the next block's Q, one block ahead (its buffer was freed by S(n-1))
           const int bn = (n + 1) & 1;
-          if (n + 1 >= 2 && !(ok = wait_bounded(&q_empty[bn], (((n + 1) >> 1) - 1) & 1, abort_flag))) break;
-          load_q(nxt, bn);
-        }
-        if (n >= 1 && !(ok = wait_bounded(v_empty, (n - 1) & 1, abort_flag))) break;
-        mbar_arrive_expect_tx(v_full, 2 * N * 128);
+          const bool next_in_pair = (blk + 1 < cur.nblk);
+          if (!next_in_pair) rn = sw_next(p, r + 1, rounds, nxt);
+          if (next_in_pair || rn >= 0) {
+            if (n + 1 >= 2 && !(ok = wait_bounded(&q_empty[bn], (((n + 1) >> 1) - 1) & 1, abort_flag))) break;
+            if (next_in_pair)
+              load_q(cur, blk + 1, bn);
+            else
+              load_q(nxt, 0, bn);
+          }
+          if (blk == 0) {
+            if (kp >= 1 && !(ok = wait_bounded(v_empty, (kp - 1) & 1, abort_flag))) break;
+            mbar_arrive_expect_tx(v_full, 2 * N * 128);
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tma_load_3d(smem + kSwOffV + c * kSwKBox, &tm_v, v_full, c * 64, cur.g, cur.b0 + k0);
+            for (int c = 0; c < 2; ++c)
+              tma_load_3d(smem + kSwOffV + c * kSwKBox, &tm_v, v_full, c * 64, cur.g, cur.b0 + k0);
+            ++kp;
+          }
+        }
         cur = nxt;
         r = rn;
       }
@@ -184,11 +202,13 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
       const uint32_t tO = tbase + 384;
       bool ok = true;
-      // O = P(m) V over N keys: N/16 MMAs (P: 8 TMEM columns each; V: 16 rows = 2 KB)
-      auto do_pv = [&](int m) {
+      // O = P(m) V over N keys: N/16 MMAs (P: 8 TMEM columns each; V: 16 rows = 2 KB).
+      // Block m is the blk-th of pair kp_m; the pair's V is waited for at its first
+      // block and released after its last.
+      auto do_pv = [&](int m, int kp_m, bool first_of_pair, bool last_of_pair) {
         const int bm = m & 1;
         if (!(ok = wait_bounded(&p_full[bm], (m >> 1) & 1, abort_flag))) return;
-        if (!(ok = wait_bounded(v_full, m & 1, abort_flag))) return;
+        if (first_of_pair && !(ok = wait_bounded(v_full, kp_m & 1, abort_flag))) return;
         if (m >= 1 && !(ok = wait_bounded(o_empty, (m - 1) & 1, abort_flag))) return;
         tc_fence_after();
         const uint32_t tP = tbase + bm * kSwNMax;
@@ -197,31 +217,39 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           umma_ts(tO, tP + kk * 8, smem_desc_sw128(aV + kk * 2048, kSwKBox, 1024), idesc_o,
                   kk > 0 ? 1u : 0u);
         umma_commit(o_full);
-        umma_commit(v_empty);
+        if (last_of_pair) umma_commit(v_empty);
       };
       SwItem it;
-      int n = 0;
-      for (int r = sw_next(p, 0, rounds, it); ok && r >= 0; r = sw_next(p, r + 1, rounds, it), ++n) {
-        const int b = n & 1;
-        if (!(ok = wait_bounded(&q_full[b], (n >> 1) & 1, abort_flag))) break;
-        if (!(ok = wait_bounded(k_full, n & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t aQ = sbase + kSwOffQ + b * kSwQBytes;
-        const uint32_t aK = sbase + kSwOffK;
-        const uint32_t tS = tbase + b * kSwNMax;
+      int n = 0, kp = 0;
+      int pm = -1, pkp = 0;     // previous block: number, pair
+      bool pfirst = false, plast = false;
+      for (int r = sw_next(p, 0, rounds, it); ok && r >= 0; r = sw_next(p, r + 1, rounds, it), ++kp) {
+        for (int blk = 0; ok && blk < it.nblk; ++blk, ++n) {
+          const int b = n & 1;
+          if (!(ok = wait_bounded(&q_full[b], (n >> 1) & 1, abort_flag))) break;
+          if (blk == 0 && !(ok = wait_bounded(k_full, kp & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t aQ = sbase + kSwOffQ + b * kSwQBytes;
+          const uint32_t aK = sbase + kSwOffK;
+          const uint32_t tS = tbase + b * kSwNMax;
 #pragma unroll
-        for (int kk = 0; kk < 12; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          umma_ss(tS, smem_desc_sw128(aQ + (kk >> 2) * 16384 + off, 16, 1024),
-                  smem_desc_sw128(aK + (kk >> 2) * kSwKBox + off, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 12; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            umma_ss(tS, smem_desc_sw128(aQ + (kk >> 2) * 16384 + off, 16, 1024),
+                    smem_desc_sw128(aK + (kk >> 2) * kSwKBox + off, 16, 1024), idesc_s,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[b]);
+          umma_commit(&q_empty[b]);
+          if (blk == it.nblk - 1) umma_commit(k_empty);
+          if (pm >= 0) do_pv(pm, pkp, pfirst, plast);
+          pm = n;
+          pkp = kp;
+          pfirst = (blk == 0);
+          plast = (blk == it.nblk - 1);
         }
-        umma_commit(&s_full[b]);
-        umma_commit(k_empty);
-        umma_commit(&q_empty[b]);
-        if (n >= 1) do_pv(n - 1);
       }
-      if (ok && n >= 1) do_pv(n - 1);
+      if (ok && pm >= 0) do_pv(pm, pkp, pfirst, plast);
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ softmax
@@ -231,11 +259,12 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     SwItem it;
     int n = 0;
     bool ok = true;
-    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it), ++n) {
+    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it))
+    for (int blk = 0; ok && blk < it.nblk; ++blk, ++n) {
       const int b = n & 1;
       const int hg = it.g * p.G + hh;
-      const int qpos = it.q0 + a;
-      const int k0 = it.q0 + p.QB - N;
+      const int qpos = it.q0 + blk * p.QB + a;
+      const int k0 = it.q0 + 2 * p.QB - N;
       const int c_hi = qpos - k0;                              // keys <= qpos
       const int c_lo = max(qpos - p.window + 1, 0) - k0;       // keys in window, >= 0
       const float sg2 = p.sinks ? p.sinks[hg] * 1.4426950408889634f : -INFINITY;
@@ -291,7 +320,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     SwItem it;
     int n = 0;
     bool ok = true;
-    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it), ++n) {
+    for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it))
+    for (int blk = 0; ok && blk < it.nblk; ++blk, ++n) {
       const int b = n & 1;
       if (!(ok = wait_bounded(o_full, n & 1, abort_flag))) break;
       tc_fence_after();
@@ -302,7 +332,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       if (!(ok = wait_bounded(&ml_full[b], (n >> 1) & 1, abort_flag))) break;
       const float2 mlv = ml[b * 128 + r];
       mbar_arrive(&ml_empty[b]);
-      const int qpos = it.q0 + a;
+      const int qpos = it.q0 + blk * p.QB + a;
       if (qpos < it.len) {
         const int tok = it.b0 + qpos;
         const int hg = it.g * p.G + hh;
