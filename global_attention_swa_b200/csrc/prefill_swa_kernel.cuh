@@ -15,14 +15,16 @@
 // With the whole window in one tile there is no online rescaling: max,
 // exponentials and the sink's share are exact for the row.
 //
-//   warp 8      TMA producer: Q double-buffered (2 x 48 KB, from DRAM, one
+//   warp 12     TMA producer: Q double-buffered (2 x 48 KB, from DRAM, one
 //               block ahead), K (N x 384 B) and V (N x 256 B) once per pair.
-//   warp 9      MMA issuer: S(n) = Q K^T into one of two TMEM score buffers,
-//               then O = P(n-1) V for the previous block (software pipelined).
-//   warps 0-3   softmax: one row per thread, two passes over the TMEM row
-//               (max, then exponentials), P written back as bf16.
-//   warps 4-7   epilogue: O / l -> bf16/fp32 rows, lse.
-//   warps 10-11 idle (complete the third warpgroup)
+//   warp 13     MMA issuer: S(n) = Q K^T into TMEM score buffer n & 1, then
+//               O = P(n-1) V for the previous block (software pipelined).
+//   warps 0-7   softmax: two warpgroups, warpgroup s takes the blocks with
+//               n & 1 == s (its own score buffer), one row per thread, two
+//               passes over the TMEM row (max, then exponentials), P written
+//               back as bf16.  Chunks of 16 columns wholly inside the row's
+//               window skip the per-element mask.
+//   warps 8-11  epilogue: O / l -> bf16/fp32 rows, lse.
 //
 // TMEM: S_0 [0, 192), S_1 [192, 384), O [384, 512).
 #pragma once
@@ -31,7 +33,7 @@
 
 namespace mimo {
 
-constexpr int kSwThreads = 384;
+constexpr int kSwThreads = 448;
 constexpr int kSwNMax = 192;
 constexpr int kSwQBytes = 3 * 16384;                   // [128 rows][192 dims] as 3 boxes
 constexpr int kSwKBox = kSwNMax * 128;                 // [N rows][64 dims], 1024-aligned
@@ -109,7 +111,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   float2* ml = reinterpret_cast<float2*>(smem + kSwOffML);  // [2][128] (m, l) per row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 8) {
+  if (warp == 12) {
     if (lane == 0) {
       for (int i = 0; i < 2; ++i) {
         mbar_init(&q_full[i], 1);
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   const int rounds = *abort_flag ? 0 : (p.num_items + gridDim.x - 1) / gridDim.x;
   const int N = p.N;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -195,7 +197,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         r = rn;
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, N, false, false);
@@ -251,17 +253,19 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       }
       if (ok && pm >= 0) do_pv(pm, pkp, pfirst, plast);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;  // TMEM lane = row = query * G + head
+    const int s = warp >> 2;                   // this warpgroup's blocks: n & 1 == s
+    const int r = (warp & 3) * 32 + lane;      // TMEM lane = row = query * G + head
     const int a = r / p.G, hh = r % p.G;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     SwItem it;
     int n = 0;
     bool ok = true;
     for (int rr = sw_next(p, 0, rounds, it); ok && rr >= 0; rr = sw_next(p, rr + 1, rounds, it))
     for (int blk = 0; ok && blk < it.nblk; ++blk, ++n) {
       const int b = n & 1;
+      if (b != s) continue;
       const int hg = it.g * p.G + hh;
       const int qpos = it.q0 + blk * p.QB + a;
       const int k0 = it.q0 + 2 * p.QB - N;
@@ -272,33 +276,53 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tc_fence_after();
       const uint32_t tS = tbase + lane_off + b * kSwNMax;
       // pass 1: row max over the visible columns
-      float mx = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16];
         tmem_load16_sync(tS + c0, v);
+        if (c0 >= c_lo && c0 + 15 <= c_hi) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = c0 + e;
-          if (c >= c_lo && c <= c_hi) mx = fmaxf(mx, __uint_as_float(v[e]));
+          for (int e = 0; e < 16; e += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+            mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = c0 + e;
+            if (c >= c_lo && c <= c_hi) mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+          }
         }
       }
-      float m = fmaxf(sg2, mx * p.scale_log2);
+      const float m = fmaxf(sg2, fmaxf(mx0, mx1) * p.scale_log2);
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same columns
       float l0 = 0.f, l1 = 0.f;
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16], pk[8];
         tmem_load16_sync(tS + c0, v);
+        if (c0 >= c_lo && c0 + 15 <= c_hi) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = c0 + 2 * e;
-          const float x0 = fmaf(__uint_as_float(v[2 * e]), p.scale_log2, neg_m);
-          const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, neg_m);
-          const float p0 = (c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f;
-          const float p1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f;
-          l0 += p0;
-          l1 += p1;
-          pk[e] = pack_bf16(p0, p1);
+          for (int e = 0; e < 8; ++e) {
+            const float2 x = fma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
+                                  make_float2(p.scale_log2, p.scale_log2), make_float2(neg_m, neg_m));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
+            l0 += p0;
+            l1 += p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = c0 + 2 * e;
+            const float x0 = fmaf(__uint_as_float(v[2 * e]), p.scale_log2, neg_m);
+            const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, neg_m);
+            const float p0 = (c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f;
+            const float p1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f;
+            l0 += p0;
+            l1 += p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
         }
         tmem_st8(tS + c0 / 2, pk);
       }
@@ -311,9 +335,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       ml[b * 128 + r] = make_float2(m, l);
       mbar_arrive(&ml_full[b]);
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ epilogue
-    const int r = threadIdx.x - 128;
+    const int r = threadIdx.x - 256;
     const int a = r / p.G, hh = r % p.G;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tO = tbase + lane_off + 384;
@@ -325,40 +349,47 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       const int b = n & 1;
       if (!(ok = wait_bounded(o_full, n & 1, abort_flag))) break;
       tc_fence_after();
-      float o[128];
-      tmem_load128_sync(tO, o);
-      tc_fence_before();
-      mbar_arrive(o_empty);
       if (!(ok = wait_bounded(&ml_full[b], (n >> 1) & 1, abort_flag))) break;
       const float2 mlv = ml[b * 128 + r];
       mbar_arrive(&ml_empty[b]);
       const int qpos = it.q0 + blk * p.QB + a;
-      if (qpos < it.len) {
-        const int tok = it.b0 + qpos;
-        const int hg = it.g * p.G + hh;
-        const float l = mlv.y;
-        const float f = (l > 0.f) ? p.v_scale / l : 0.f;
-        const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
+      const bool live = qpos < it.len;
+      const int tok = it.b0 + qpos;
+      const int hg = it.g * p.G + hh;
+      const float l = mlv.y;
+      const float f = (l > 0.f) ? p.v_scale / l : 0.f;
+      const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
+      // O in two 64-column halves (registers: 448 threads leave 128 per thread);
+      // O is released to the next P.V after the second half is in registers.
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float o[64];
+        tmem_load64_sync(tO + h * 64, o);
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(o_empty);
+        }
+        if (!live) continue;
         if (p.out_f32) {
-          float* dst = reinterpret_cast<float*>(p.out) + ob;
+          float* dst = reinterpret_cast<float*>(p.out) + ob + h * 64;
           if (p.out_v8) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
+            for (int e = 0; e < 8; ++e)
               st_global_v8(dst + 8 * e, __float_as_uint(o[8 * e] * f), __float_as_uint(o[8 * e + 1] * f),
                            __float_as_uint(o[8 * e + 2] * f), __float_as_uint(o[8 * e + 3] * f),
                            __float_as_uint(o[8 * e + 4] * f), __float_as_uint(o[8 * e + 5] * f),
                            __float_as_uint(o[8 * e + 6] * f), __float_as_uint(o[8 * e + 7] * f));
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
+            for (int e = 0; e < 16; ++e)
               reinterpret_cast<float4*>(dst)[e] =
                   make_float4(o[4 * e] * f, o[4 * e + 1] * f, o[4 * e + 2] * f, o[4 * e + 3] * f);
           }
         } else {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ob;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + ob + h * 64;
           if (p.out_v8) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
+            for (int e = 0; e < 4; ++e)
               st_global_v8(dst + 16 * e, pack_bf16(o[16 * e + 0] * f, o[16 * e + 1] * f),
                            pack_bf16(o[16 * e + 2] * f, o[16 * e + 3] * f),
                            pack_bf16(o[16 * e + 4] * f, o[16 * e + 5] * f),
@@ -369,7 +400,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
                            pack_bf16(o[16 * e + 14] * f, o[16 * e + 15] * f));
           } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 8; ++e) {
               uint4 u;
               u.x = pack_bf16(o[8 * e + 0] * f, o[8 * e + 1] * f);
               u.y = pack_bf16(o[8 * e + 2] * f, o[8 * e + 3] * f);
@@ -379,6 +410,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
             }
           }
         }
+      }
+      if (live) {
         if (p.lse)
           p.lse[(size_t)hg * p.total + tok] =
               (l > 0.f) ? (mlv.x * 0.6931471805599453f + logf(l)) : -INFINITY;
@@ -388,7 +421,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
