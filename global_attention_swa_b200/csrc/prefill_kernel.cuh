@@ -226,22 +226,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
       const uint32_t tS0 = tbase + 0, tS1 = tbase + 128, tO0 = tbase + 256, tO1 = tbase + 384;
-      const uint32_t aQ0 = sbase + kPfOffQ0, aQ1 = sbase + kPfOffQ1;
+      // Descriptors as one shared high word plus a low word per operand; the
+      // per-MMA offsets below are compile-time constants (address units of 16 B).
+      constexpr uint32_t dhi = desc_hi_sw128(1024);
+      const uint32_t dQ0 = desc_lo_sw128(sbase + kPfOffQ0, 16), dQ1 = desc_lo_sw128(sbase + kPfOffQ1, 16);
+      const uint32_t dK0 = desc_lo_sw128(sbase + kPfOffK, 16);
+      const uint32_t dV = desc_lo_sw128(sbase + kPfOffV, 16384);
       // S_i = Q_i K^T over 192 dims = 12 MMAs of K=16 (3 swizzle boxes x 4 steps of 32 B)
-      auto issue_s = [&](uint32_t tS, uint32_t aQ, uint32_t aK) {
+      auto issue_s = [&](uint32_t tS, uint32_t dQ, uint32_t dK) {
 #pragma unroll
         for (int kk = 0; kk < 12; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tS, kmajor_desc(aQ + off), kmajor_desc(aK + off), idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_ss_lo(tS, dQ + off, dK + off, dhi, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
       // O_i += P_i V over 128 keys = 8 MMAs of K=16 (P: 8 TMEM columns each; V: 16 rows = 2 KB)
       auto issue_pv = [&](uint32_t tO, uint32_t tP, bool acc) {
-        const uint32_t aV = sbase + kPfOffV;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tO, tP + kk * 8, mnmajor_desc(aV + kk * 2048), idesc_o, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_lo(tO, tP + kk * 8, dV + ((kk * 2048) >> 4), dhi, idesc_o, (acc || kk > 0) ? 1u : 0u);
       };
+      auto dK = [&](int stage) { return dK0 + static_cast<uint32_t>(stage) * (kPfKBytes >> 4); };
       int n = 0;           // items
       int n1 = 0;          // items with a second head
       int kt = 0;          // key tiles (all items): K ring and V phases
@@ -256,11 +261,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!(ok = wait_bounded(&k_full[kt & 1], (kt >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         {
-          const uint32_t aK = sbase + kPfOffK + (kt & 1) * kPfKBytes;
-          issue_s(tS0, aQ0, aK);
+          issue_s(tS0, dQ0, dK(kt & 1));
           umma_commit(&s_full[0]);
           if (it.has1) {
-            issue_s(tS1, aQ1, aK);
+            issue_s(tS1, dQ1, dK(kt & 1));
             umma_commit(&s_full[1]);
           }
           umma_commit(&k_empty[kt & 1]);
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!last) {
             if (!(ok = wait_bounded(&k_full[kn & 1], (kn >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            issue_s(tS0, aQ0, sbase + kPfOffK + (kn & 1) * kPfKBytes);
+            issue_s(tS0, dQ0, dK(kn & 1));
             umma_commit(&s_full[0]);
             if (!it.has1 && t + 1 == it.n_kt - 1) umma_commit(q_empty);
           }
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           umma_commit(v_empty);
           if (!last) {
             if (it.has1) {
-              issue_s(tS1, aQ1, sbase + kPfOffK + (kn & 1) * kPfKBytes);
+              issue_s(tS1, dQ1, dK(kn & 1));
               umma_commit(&s_full[1]);
               if (t + 1 == it.n_kt - 1) umma_commit(q_empty);
             }
