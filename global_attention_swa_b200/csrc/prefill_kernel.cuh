@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
         if (full_tile) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmax3(mx8[c & 7], s[2 * c], s[2 * c + 1]);
         } else {
           const int hi_k = qpos - kpos0;                                  // keys <= hi_k visible
           const int lo_k = p.window > 0 ? qpos - p.window + 1 - kpos0 : -1;  // keys >= lo_k visible
@@ -356,8 +356,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
           }
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
         const float m_new = fmaxf(m, mx * p.scale_log2);
         float alpha = 1.f;
         bool rescale_o = false;

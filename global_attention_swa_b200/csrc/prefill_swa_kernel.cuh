@@ -282,9 +282,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         tmem_load16_sync(tS + c0, v);
         if (c0 >= c_lo && c0 + 15 <= c_hi) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(v[e]));
-            mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
+          for (int e = 0; e < 16; e += 4) {
+            mx0 = fmax3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
         } else {
 #pragma unroll
