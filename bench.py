@@ -81,6 +81,14 @@ def decode_work(lengths, window, capacity):
     return flops, byts
 
 
+def decode_fp8_work(lengths, window, capacity):
+    """decode_work with one byte per cache element (e4m3) plus the 2 x Hkv fp32 scales."""
+    flops, byts = decode_work(lengths, window, capacity)
+    ring = window > 0 and capacity == window
+    vis = [min(L, capacity) if ring else (min(L, window) if window > 0 else L) for L in lengths]
+    return flops, byts - sum(vis) * KV_BYTES_PER_TOKEN // 2 + 2 * HKV * 4
+
+
 def floor_s(flops, byts, peaks):
     return max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
 
@@ -491,9 +499,18 @@ def run_case(args):
             # smaller caches (for profiler captures): lengths ~U[1024, cap]
             cap = args.decode_cap
             lengths = W.lengths_uniform(0, 64, 1024, cap)
-        d = W.decode_inputs(lengths, cap, window, seed=3, device=dev)
-        fn = lambda: mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks)  # noqa: E731
-        work = decode_work(lengths, window, cap)
+        if args.case == "decode_global_fp8":
+            window, cap = 0, (args.decode_cap or W.DECODE_GA_CAPACITY)
+            if args.decode_cap:
+                lengths = W.lengths_uniform(0, 64, 1024, cap)
+            d = W.decode_inputs_fp8(lengths, cap, window, seed=3, device=dev)
+            fn = lambda: mimo.mimo_attn_decode_fp8(d.q, d.k_codes, d.v_codes, d.k_scale,  # noqa: E731
+                                                   d.v_scale_kv, d.seqlens, window, d.sinks)
+            work = decode_fp8_work(lengths, window, cap)
+        else:
+            d = W.decode_inputs(lengths, cap, window, seed=3, device=dev)
+            fn = lambda: mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks)  # noqa: E731
+            work = decode_work(lengths, window, cap)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -525,11 +542,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=["step", "prefill_swa", "prefill_global", "decode_global",
-                                       "decode_ring"], default="step",
+                                       "decode_ring", "decode_global_fp8"], default="step",
                     help="run one kernel alone (profiling); 'step' is the benchmark")
     ap.add_argument("--seq-len", type=int, default=T_PREFILL, help="prefill length for --case")
     ap.add_argument("--decode-cap", type=int, default=0,
-                    help="decode_global --case with caches of this capacity (0: 262144)")
+                    help="decode_global(_fp8) --case with caches of this capacity (0: 262144)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -40,6 +40,8 @@ EXPORTED = (
     "mimo_attn_last_error",
     "mimo_attn_device_status",
     "mimo_attn_decode_noalloc",
+    "mimo_attn_decode_fp8_workspace_size",
+    "mimo_attn_decode_fp8",
 )
 
 
@@ -78,6 +80,11 @@ def _load():
     lib.mimo_attn_last_error.restype = ctypes.c_char_p
     lib.mimo_attn_device_status.argtypes = [vp]
     lib.mimo_attn_device_status.restype = i32
+    lib.mimo_attn_decode_fp8_workspace_size.argtypes = [dp, i32, i32, i32]
+    lib.mimo_attn_decode_fp8_workspace_size.restype = sz
+    lib.mimo_attn_decode_fp8.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp,
+                                         sz, vp]
+    lib.mimo_attn_decode_fp8.restype = i32
     return lib
 
 
@@ -158,6 +165,35 @@ def mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, out=None, lse=
     _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                 _ptr(seqlens), B, C, int(window), _ptr(sinks), _ptr(out),
                                 _ptr(lse), _ptr(workspace), wbytes, _stream(stream)))
+    return out, lse
+
+
+def mimo_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale_kv, seqlens, window, sinks,
+                         out=None, lse=None, workspace=None, out_dtype=torch.bfloat16,
+                         softmax_scale=None, v_scale=1.0, return_lse=True, stream=None):
+    """One decode step against e4m3 caches.  q [B,Hq,192] bf16; caches [B,C,Hkv,192/128]
+    as torch.float8_e4m3fn or uint8 codes; k_scale / v_scale_kv [Hkv] fp32.
+
+    Returns (out [B,Hq,128], lse [B,Hq] fp32 or None).
+    """
+    B, hq, dqk = q.shape
+    C, hkv = k_cache.shape[1], k_cache.shape[2]
+    dv = v_cache.shape[3]
+    if k_cache.element_size() != 1 or v_cache.element_size() != 1:
+        raise TypeError("FP8 caches hold one byte per element")
+    if out is None:
+        out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
+    need = int(lib.mimo_attn_decode_fp8_workspace_size(ctypes.byref(dims), B, C, int(window)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.mimo_attn_decode_fp8(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(k_scale), _ptr(v_scale_kv), _ptr(seqlens), B, C,
+                                    int(window), _ptr(sinks), _ptr(out), _ptr(lse),
+                                    _ptr(workspace), wbytes, _stream(stream)))
     return out, lse
 
 

@@ -423,4 +423,43 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int col_bf16) {
   return static_cast<uint32_t>(row * 128 + (((chunk ^ (row & 7)) << 4) | ((col_bf16 & 7) << 1)));
 }
 
+// C[16x8] += A[16x16] * B[16x8], f16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The two e4m3 bytes of the low (hi = false) or high half of x as an f16 pair
+// (the lower byte becomes the lower half).  Exact: every e4m3 value is an f16.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x, bool hi) {
+  uint32_t r;
+  const uint16_t h = static_cast<uint16_t>(hi ? (x >> 16) : (x & 0xFFFFu));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+  return r;
+}
+
+// Byte permute: result byte i = byte (sel >> 4i) & 7 of {b, a} (a = bytes 0-3).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte offset of (row, byte column) in a TMA box with 64-byte rows and
+// 64-byte swizzle (16-byte chunk index XOR bits 7..8 of the address).
+__device__ __forceinline__ uint32_t sw64_offset(int row, int col_byte) {
+  const int chunk = col_byte >> 4;
+  return static_cast<uint32_t>(row * 64 + (((chunk ^ ((row >> 1) & 3)) << 4) | (col_byte & 15)));
+}
+
 }  // namespace mimo

@@ -48,6 +48,8 @@ struct DecodeParams {
   float scale_log2;  // softmax_scale * log2(e)
   float v_scale;
   int out_f32;
+  const float* k_scale;     // [Hkv] FP8 caches only: K value = code * k_scale[g]
+  const float* kv_v_scale;  // [Hkv] FP8 caches only: V value = code * kv_v_scale[g]; null = 1
 };
 
 // Visible slot range [lo, hi) of sequence b (see mimo_attn.h).
@@ -337,7 +339,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 // Merge the split partials of every (b, query head) and fold the sink:
 //   M = max(sigma, max_c m_c),  Z = 2^(sigma-M) + sum_c 2^(m_c-M) l_c,
-//   out = v_scale * sum_c 2^(m_c-M) o_c / Z,   lse = ln Z + M ln 2.
+//   out = v_scale * sum_c 2^(m_c-M) o_c / Z,   lse = ln Z + M ln 2
+// (times the V scale of the KV head for FP8 caches, whose partials are in code units).
 // One warp per (b, h); lane handles 4 of the 128 value columns.
 __global__ void __launch_bounds__(256)
     decode_combine_kernel(const DecodeParams p) {
@@ -369,7 +372,8 @@ __global__ void __launch_bounds__(256)
       acc.w += w * oc.w;
     }
   }
-  const float f = (Z > 0.f) ? p.v_scale / Z : 0.f;
+  const float vs = p.kv_v_scale ? p.kv_v_scale[g] : 1.f;
+  const float f = (Z > 0.f) ? p.v_scale * vs / Z : 0.f;
   const size_t ob = ((size_t)b * p.Hq + h) * 128 + lane * 4;
   if (p.out_f32) {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob) =

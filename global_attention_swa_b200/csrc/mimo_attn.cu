@@ -13,6 +13,7 @@
 #include "../../include/mimo_attn.h"
 #include "common.cuh"
 #include "decode_kernel.cuh"
+#include "decode_fp8_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
@@ -61,7 +62,9 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor with `rank` dims (innermost first), byte strides of dims 1.., box sizes.
 mimo_status_t make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                       const uint64_t* strides_bytes, const uint32_t* box) {
+                       const uint64_t* strides_bytes, const uint32_t* box,
+                       CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MIMO_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   cuuint64_t gd[5], gs[4];
@@ -72,8 +75,8 @@ mimo_status_t make_map(CUtensorMap* map, const void* base, int rank, const uint6
     es[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bd,
-                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, dtype, rank, const_cast<void*>(base), gd, gs, bd,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MIMO_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MIMO_OK;
@@ -135,6 +138,11 @@ mimo_status_t ensure_attributes() {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kDecSmemBytes),
                        "decode smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_fp8_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kD8SmemBytes),
+                       "FP8 decode smem attribute")))
     return st;
   done[dev] = true;
   return MIMO_OK;
@@ -331,11 +339,17 @@ size_t mimo_attn_decode_workspace_size(const mimo_attn_dims_t* dims, int batch, 
                             decode_plan(batch, dims->num_heads_kv, capacity, window));
 }
 
-mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, const void* k_cache,
-                               const void* v_cache, const int32_t* seqlens, int batch,
-                               int capacity, int window, const float* sinks, void* out,
-                               float* lse, void* workspace, size_t workspace_bytes,
-                               void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Decode over a bf16 cache (fp8 = false) or an e4m3 cache with per-KV-head
+// scales (fp8 = true); both entry points validate and launch here.
+mimo_status_t decode_impl(const mimo_attn_dims_t* dims, const void* q, const void* k_cache,
+                          const void* v_cache, bool fp8, const float* k_scale,
+                          const float* v_scale_kv, const int32_t* seqlens, int batch,
+                          int capacity, int window, const float* sinks, void* out, float* lse,
+                          void* workspace, size_t workspace_bytes, void* stream) {
   mimo_status_t st = check_dims(dims);
   if (st) return st;
   if (window < 0) return fail(MIMO_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
@@ -347,6 +361,10 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, cons
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       (lse && ((uintptr_t)lse & 3u)) || (sinks && ((uintptr_t)sinks & 3u)))
     return fail(MIMO_ERR_INVALID_ARG, "q, caches and out must be 16-byte aligned");
+  if (fp8 && (!k_scale || !v_scale_kv))
+    return fail(MIMO_ERR_INVALID_ARG, "an FP8 cache needs k_scale and v_scale_kv");
+  if (fp8 && (((uintptr_t)k_scale & 3u) || ((uintptr_t)v_scale_kv & 3u)))
+    return fail(MIMO_ERR_INVALID_ARG, "k_scale and v_scale_kv must be 4-byte aligned");
   const int Hq = dims->num_heads_q, Hkv = dims->num_heads_kv, G = Hq / Hkv;
   if (G > 16) return fail(MIMO_ERR_UNSUPPORTED, "decode packs at most 16 query heads per KV head (got %d)", G);
   if ((long)batch * capacity > 0x7fffffffL)
@@ -362,16 +380,23 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, cons
 
   CUtensorMap tk, tv;
   {
-    const uint64_t d[2] = {(uint64_t)Hkv * 192, (uint64_t)batch * capacity};
-    const uint64_t s[1] = {(uint64_t)Hkv * 192 * 2};
-    const uint32_t b[2] = {64, (uint32_t)mimo::kDecTileKeys};
-    if ((st = make_map(&tk, k_cache, 2, d, s, b))) return st;
-  }
-  {
-    const uint64_t d[2] = {(uint64_t)Hkv * 128, (uint64_t)batch * capacity};
-    const uint64_t s[1] = {(uint64_t)Hkv * 128 * 2};
-    const uint32_t b[2] = {64, (uint32_t)mimo::kDecTileKeys};
-    if ((st = make_map(&tv, v_cache, 2, d, s, b))) return st;
+    // bf16: boxes of 64 elements (128 B, 128-byte swizzle); e4m3: 64 bytes, 64-byte swizzle
+    const int eb = fp8 ? 1 : 2;
+    const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle sw = fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint32_t rows = fp8 ? (uint32_t)mimo::kD8TileKeys : (uint32_t)mimo::kDecTileKeys;
+    {
+      const uint64_t d[2] = {(uint64_t)Hkv * 192, (uint64_t)batch * capacity};
+      const uint64_t s[1] = {(uint64_t)Hkv * 192 * eb};
+      const uint32_t b[2] = {64, rows};
+      if ((st = make_map(&tk, k_cache, 2, d, s, b, dt, sw))) return st;
+    }
+    {
+      const uint64_t d[2] = {(uint64_t)Hkv * 128, (uint64_t)batch * capacity};
+      const uint64_t s[1] = {(uint64_t)Hkv * 128 * eb};
+      const uint32_t b[2] = {64, rows};
+      if ((st = make_map(&tv, v_cache, 2, d, s, b, dt, sw))) return st;
+    }
   }
   mimo::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -394,9 +419,15 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, cons
   p.scale_log2 = scale_log2_of(dims);
   p.v_scale = v_scale_of(dims);
   p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+  p.k_scale = fp8 ? k_scale : nullptr;
+  p.kv_v_scale = fp8 ? v_scale_kv : nullptr;
   dim3 grid(pl.nsplit, Hkv, batch);
-  mimo::decode_split_kernel<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, (cudaStream_t)stream>>>(
-      tk, tv, p);
+  if (fp8)
+    mimo::decode_split_fp8_kernel<<<grid, mimo::kD8Threads, mimo::kD8SmemBytes, (cudaStream_t)stream>>>(
+        tk, tv, p);
+  else
+    mimo::decode_split_kernel<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, (cudaStream_t)stream>>>(
+        tk, tv, p);
   if ((st = cuda_check(cudaGetLastError(), "decode launch"))) return st;
   if (pl.nsplit > 1) {
     const int warps = batch * Hq;
@@ -405,6 +436,34 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, cons
     if ((st = cuda_check(cudaGetLastError(), "decode combine launch"))) return st;
   }
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* seqlens, int batch,
+                               int capacity, int window, const float* sinks, void* out,
+                               float* lse, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return decode_impl(dims, q, k_cache, v_cache, false, nullptr, nullptr, seqlens, batch, capacity,
+                     window, sinks, out, lse, workspace, workspace_bytes, stream);
+}
+
+size_t mimo_attn_decode_fp8_workspace_size(const mimo_attn_dims_t* dims, int batch, int capacity,
+                                           int window) {
+  return mimo_attn_decode_workspace_size(dims, batch, capacity, window);
+}
+
+mimo_status_t mimo_attn_decode_fp8(const mimo_attn_dims_t* dims, const void* q,
+                                   const void* k_cache, const void* v_cache,
+                                   const float* k_scale, const float* v_scale_kv,
+                                   const int32_t* seqlens, int batch, int capacity, int window,
+                                   const float* sinks, void* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return decode_impl(dims, q, k_cache, v_cache, true, k_scale, v_scale_kv, seqlens, batch,
+                     capacity, window, sinks, out, lse, workspace, workspace_bytes, stream);
 }
 
 mimo_status_t mimo_attn_device_status(void* stream) {

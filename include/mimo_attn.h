@@ -137,6 +137,40 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q,
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace bytes for mimo_attn_decode_fp8 (the same split plan as the bf16
+ * decode, so the same size).
+ */
+size_t mimo_attn_decode_fp8_workspace_size(const mimo_attn_dims_t* dims,
+                                           int batch, int capacity, int window);
+
+/*
+ * One decode step against an FP8 KV cache (MiMo-V2-Flash model doc, "Key
+ * features": FP8 mixed precision; the cache format is this library's own).
+ *
+ *   k_cache    [batch, capacity, Hkv, Dqk] e4m3 bytes (OCP FP8 E4M3: sign,
+ *              4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ *              S.1111.111 = NaN, largest finite 448)
+ *   v_cache    [batch, capacity, Hkv, Dv ] e4m3 bytes
+ *   k_scale    [Hkv] fp32 on the device: key element = code * k_scale[g]
+ *   v_scale_kv [Hkv] fp32 on the device: value element = code * v_scale_kv[g]
+ *              (g = the key/value head; one pair of scales per layer and head)
+ *
+ * Every other argument, the ring/linear cache rules, the workspace and the
+ * error behaviour are those of mimo_attn_decode.  The products run in f16
+ * with fp32 accumulation: e4m3 codes convert to f16 exactly, q is rounded to
+ * f16 once (q elements must lie within the f16 range, |q| < 65504), and the
+ * softmax weights are rounded to f16 for the P.V product.  k_scale and
+ * v_scale_kv must be non-NULL and 4-byte aligned (else MIMO_ERR_INVALID_ARG).
+ */
+mimo_status_t mimo_attn_decode_fp8(const mimo_attn_dims_t* dims, const void* q,
+                                   const void* k_cache, const void* v_cache,
+                                   const float* k_scale, const float* v_scale_kv,
+                                   const int32_t* seqlens, int batch, int capacity,
+                                   int window, const float* sinks, void* out,
+                                   float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
  * mimo_attn_decode without a workspace and without allocating.  The model
  * documentation has no counterpart to this call: it exists for callers that
  * cannot call cudaMalloc -- code running in a process whose device memory is

@@ -12,6 +12,9 @@ Modules
 -------
 ``attention``  vectorised fp64 prefill and decode (NumPy matmuls per query block).
 ``brute``      scalar triple loops for tiny shapes, used to pin ``attention``.
+``fp8``        e4m3 decoding from the format's definition and decode over FP8
+               KV caches with per-KV-head scales (``attention.decode`` on the
+               dequantised caches).
 
 Every function here is pinned by a ``-m "not gpu"`` test against something
 other than itself (brute force, closed forms, a library special case, or the

@@ -90,6 +90,34 @@ def test_ring_decode_needs_no_workspace():
     assert mimo.mimo_attn_decode_workspace_size(64, 4, 64, 129, 129) == 0
 
 
+def _decode_fp8(dims, batch=2, cap=1024, window=0, ks=FAKE, vs=FAKE, ws=None, ws_bytes=0, q=FAKE):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    return mimo.lib.mimo_attn_decode_fp8(ctypes.byref(dims), p(q), p(FAKE), p(FAKE), p(ks), p(vs),
+                                         p(FAKE), batch, cap, window, None, p(FAKE), None, p(ws),
+                                         ws_bytes, None)
+
+
+def test_decode_fp8_rejects_bad_arguments():
+    assert _decode_fp8(_dims(), ks=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert "k_scale" in mimo.lib.mimo_attn_last_error().decode()
+    assert _decode_fp8(_dims(), vs=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode_fp8(_dims(), ks=FAKE + 2) == mimo.MIMO_ERR_INVALID_ARG   # misaligned scales
+    assert _decode_fp8(_dims(), window=-1) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode_fp8(_dims(), q=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _decode_fp8(_dims(dqk=128)) == mimo.MIMO_ERR_UNSUPPORTED
+    assert _decode_fp8(_dims(), batch=0) == mimo.MIMO_OK
+
+
+def test_decode_fp8_workspace_matches_bf16_plan():
+    for args in ((64, 4, 64, 262144, 0), (64, 4, 64, 129, 129), (16, 1, 3, 5000, 0)):
+        dims = mimo.make_dims(args[0], args[1])
+        assert (mimo.lib.mimo_attn_decode_fp8_workspace_size(ctypes.byref(dims), *args[2:])
+                == mimo.mimo_attn_decode_workspace_size(*args))
+    need = mimo.mimo_attn_decode_workspace_size(64, 4, 64, 262144, 0)
+    assert _decode_fp8(_dims(), batch=64, cap=262144, ws=None) == mimo.MIMO_ERR_WORKSPACE
+    assert _decode_fp8(_dims(), batch=64, cap=262144, ws=FAKE, ws_bytes=need - 16) == mimo.MIMO_ERR_WORKSPACE
+
+
 def test_last_error_is_empty_after_success():
     assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
     assert mimo.lib.mimo_attn_last_error().decode() == ""

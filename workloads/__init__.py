@@ -14,6 +14,10 @@ Recipe (shapes from ``MiMoV2FlashConfig``: 64 query heads, 4 key/value heads,
 * decode caches: slots holding tokens that exist are ~N(0, 1); slots past a
   sequence's length are filled with NaN ("poison") unless ``poison=False`` so
   that any read of an invalid slot shows up in the output.
+* FP8 decode caches: the same N(0, 1) draws divided by a fixed per-KV-head
+  scale (K: (8 + g) / 448, V: (6 + 2 g) / 448, so about +-8 sigma spans the
+  e4m3 range), clamped to +-448 and rounded to e4m3 by torch's float8_e4m3fn
+  cast; poison slots hold the NaN code 0x7F.
 """
 
 from __future__ import annotations
@@ -115,6 +119,54 @@ def decode_inputs(seqlens, capacity, window, hq=HQ, hkv=HKV, dqk=DQK, dv=DV,
     s = torch.randn(hq, generator=g, dtype=torch.float32, device=device) if sinks else None
     sl = torch.tensor([int(L) for L in seqlens], dtype=torch.int32, device=device)
     return DecodeInputs(q, k, v, sl, s, window, capacity)
+
+
+@dataclass
+class DecodeInputsFp8:
+    q: torch.Tensor
+    k_codes: torch.Tensor    # uint8 e4m3 codes [B, C, Hkv, Dqk]
+    v_codes: torch.Tensor    # uint8 e4m3 codes [B, C, Hkv, Dv]
+    k_scale: torch.Tensor    # [Hkv] fp32
+    v_scale_kv: torch.Tensor  # [Hkv] fp32
+    seqlens: torch.Tensor
+    sinks: torch.Tensor | None
+    window: int
+    capacity: int
+
+
+def fp8_kv_scales(hkv=HKV, device="cpu"):
+    """Fixed per-KV-head cache scales (K, V) used by the FP8 decode workloads."""
+    k = torch.tensor([(8.0 + g) / 448.0 for g in range(hkv)], dtype=torch.float32, device=device)
+    v = torch.tensor([(6.0 + 2.0 * g) / 448.0 for g in range(hkv)], dtype=torch.float32, device=device)
+    return k, v
+
+
+def _e4m3_codes(x, scale):
+    y = (x / scale.view(1, -1, 1)).clamp_(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def decode_inputs_fp8(seqlens, capacity, window, hq=HQ, hkv=HKV, dqk=DQK, dv=DV,
+                      seed=0, sinks=True, poison=True, device="cpu"):
+    """One decode step over e4m3 caches: q [B,Hq,Dqk] bf16, uint8 codes, per-head scales."""
+    B = len(seqlens)
+    g = _gen(seed, device)
+    q = randn_bf16((B, hq, dqk), g, device)
+    ks, vs = fp8_kv_scales(hkv, device)
+    k = torch.empty((B, capacity, hkv, dqk), dtype=torch.uint8, device=device)
+    v = torch.empty((B, capacity, hkv, dv), dtype=torch.uint8, device=device)
+    for b, L in enumerate(seqlens):
+        n = min(int(L), capacity)
+        k[b, :n] = _e4m3_codes(torch.randn((n, hkv, dqk), generator=g, dtype=torch.float32,
+                                           device=device), ks)
+        v[b, :n] = _e4m3_codes(torch.randn((n, hkv, dv), generator=g, dtype=torch.float32,
+                                           device=device), vs)
+        if n < capacity:
+            k[b, n:] = 0x7F if poison else 0
+            v[b, n:] = 0x7F if poison else 0
+    s = torch.randn(hq, generator=g, dtype=torch.float32, device=device) if sinks else None
+    sl = torch.tensor([int(L) for L in seqlens], dtype=torch.int32, device=device)
+    return DecodeInputsFp8(q, k, v, ks, vs, sl, s, window, capacity)
 
 
 # The five workloads, by what they are.
