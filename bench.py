@@ -287,6 +287,39 @@ def run_ours(args, rank, world, peaks, peak_kind):
         e2e = run_e2e(args, mimo, swa, ga, dga, dsw, lengths, dev, floor_step_ms, world,
                       o_swa, o_ga, o_dga, o_dsw, l_swa, l_ga, l_dga, l_dsw, ws_ga, ws_sw)
 
+    # --- the next row outside the step: global decode over e4m3 caches (same
+    # lengths and capacity), timed alone after the step's region
+    extra = None
+    if not args.no_extra:
+        del dga
+        torch.cuda.empty_cache()
+        d8 = W.decode_inputs_fp8(lengths, W.DECODE_GA_CAPACITY, 0, seed=seed + 3, device=dev)
+        o8 = torch.empty_like(o_dga)
+        l8 = torch.empty_like(l_dga)
+        fn = lambda: mimo.mimo_attn_decode_fp8(d8.q, d8.k_codes, d8.v_codes, d8.k_scale,  # noqa: E731
+                                               d8.v_scale_kv, d8.seqlens, 0, d8.sinks, out=o8,
+                                               lse=l8, workspace=ws_ga)
+        ms8 = []
+        for i in range(args.warmup + 10):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms8.append(e0.elapsed_time(e1))
+        mimo.mimo_attn_device_status()
+        f8, b8 = decode_fp8_work(lengths, 0, W.DECODE_GA_CAPACITY)
+        m8 = float(np.mean(ms8))
+        extra = {"decode_global_fp8_B64_cap262144": {
+            "ms": round(m8, 4), "GB/s": round(b8 / (m8 * 1e-3) / 1e9, 1),
+            "roofline_frac": round(1e3 * floor_s(f8, b8, peaks) / m8, 4), "bound": "hbm",
+            "algorithmic_bytes": b8, "launches": 2,
+            "note": "e4m3 K/V caches with per-KV-head scales (the next row after the step's "
+                    "kernels); not part of the step or its value"}}
+        del d8
+
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
@@ -303,6 +336,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
                    "floor_ms_per_step": round(floor_step_ms, 4),
                    "peaks": {**peaks, "source": peak_kind}},
         "parts": parts,
+        "extra": extra,
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -541,6 +575,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the FP8-cache decode measured after the step")
     ap.add_argument("--case", choices=["step", "prefill_swa", "prefill_global", "decode_global",
                                        "decode_ring", "decode_global_fp8"], default="step",
                     help="run one kernel alone (profiling); 'step' is the benchmark")

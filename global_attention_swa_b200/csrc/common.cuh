@@ -433,13 +433,15 @@ __device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// The two e4m3 bytes of the low (hi = false) or high half of x as an f16 pair
-// (the lower byte becomes the lower half).  Exact: every e4m3 value is an f16.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t x, bool hi) {
-  uint32_t r;
-  const uint16_t h = static_cast<uint16_t>(hi ? (x >> 16) : (x & 0xFFFFu));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
-  return r;
+// The four e4m3 bytes of x as two f16 pairs: lo = bytes 0-1, hi = bytes 2-3 (the lower
+// byte of each pair becomes the lower half).  Exact: every e4m3 value is an f16.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
 }
 
 // Byte permute: result byte i = byte (sel >> 4i) & 7 of {b, a} (a = bytes 0-3).

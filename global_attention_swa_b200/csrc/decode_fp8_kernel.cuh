@@ -146,10 +146,15 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
           const int col = 32 * i + lcol;  // byte column within the 192-byte key row
           uint32_t x0, x1, x2, x3;
           ldsm_x4(kb + (col >> 6) * kD8BoxBytes + sw64_offset(lrow, col & 63), x0, x1, x2, x3);
-          mma_f16_16816(s[0], qa[2 * i], e4m3x2_to_f16x2(x0, false), e4m3x2_to_f16x2(x0, true));
-          mma_f16_16816(s[1], qa[2 * i], e4m3x2_to_f16x2(x1, false), e4m3x2_to_f16x2(x1, true));
-          mma_f16_16816(s[0], qa[2 * i + 1], e4m3x2_to_f16x2(x2, false), e4m3x2_to_f16x2(x2, true));
-          mma_f16_16816(s[1], qa[2 * i + 1], e4m3x2_to_f16x2(x3, false), e4m3x2_to_f16x2(x3, true));
+          uint32_t b[8];
+          e4m3x4_to_f16x2x2(x0, b[0], b[1]);
+          e4m3x4_to_f16x2x2(x1, b[2], b[3]);
+          e4m3x4_to_f16x2x2(x2, b[4], b[5]);
+          e4m3x4_to_f16x2x2(x3, b[6], b[7]);
+          mma_f16_16816(s[0], qa[2 * i], b[0], b[1]);
+          mma_f16_16816(s[1], qa[2 * i], b[2], b[3]);
+          mma_f16_16816(s[0], qa[2 * i + 1], b[4], b[5]);
+          mma_f16_16816(s[1], qa[2 * i + 1], b[6], b[7]);
         }
         // ---- scale to base 2 and mask keys past the split's end
         float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -186,12 +191,15 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
           l0 = l0 * a0 + ((p00 + p01) + (p10 + p11));
           l1 = l1 * a1 + ((p02 + p03) + (p12 + p13));
         }
+        // rescale O only when some row's running max moved (2^0 is exactly 1)
+        if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          o[n][0] *= a0;
-          o[n][1] *= a0;
-          o[n][2] *= a1;
-          o[n][3] *= a1;
+          for (int n = 0; n < 16; ++n) {
+            o[n][0] *= a0;
+            o[n][1] *= a0;
+            o[n][2] *= a1;
+            o[n][3] *= a1;
+          }
         }
         // ---- O += P V: 4 groups of 32 dims; matrices 0/1 = keys +0..7 / +8..15 of
         // dims +0..15, matrices 2/3 the same keys of dims +16..31.
@@ -211,10 +219,15 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
           x1 = prmt(x1, 0u, 0x3120u);
           x2 = prmt(x2, 0u, 0x3120u);
           x3 = prmt(x3, 0u, 0x3120u);
-          mma_f16_16816(o[4 * i + 0], pa, e4m3x2_to_f16x2(x0, false), e4m3x2_to_f16x2(x1, false));
-          mma_f16_16816(o[4 * i + 1], pa, e4m3x2_to_f16x2(x0, true), e4m3x2_to_f16x2(x1, true));
-          mma_f16_16816(o[4 * i + 2], pa, e4m3x2_to_f16x2(x2, false), e4m3x2_to_f16x2(x3, false));
-          mma_f16_16816(o[4 * i + 3], pa, e4m3x2_to_f16x2(x2, true), e4m3x2_to_f16x2(x3, true));
+          uint32_t e0[2], e1[2], e2[2], e3[2];  // [0]: dim 2c pairs, [1]: dim 2c+1 pairs
+          e4m3x4_to_f16x2x2(x0, e0[0], e0[1]);
+          e4m3x4_to_f16x2x2(x1, e1[0], e1[1]);
+          e4m3x4_to_f16x2x2(x2, e2[0], e2[1]);
+          e4m3x4_to_f16x2x2(x3, e3[0], e3[1]);
+          mma_f16_16816(o[4 * i + 0], pa, e0[0], e1[0]);
+          mma_f16_16816(o[4 * i + 1], pa, e0[1], e1[1]);
+          mma_f16_16816(o[4 * i + 2], pa, e2[0], e3[0]);
+          mma_f16_16816(o[4 * i + 3], pa, e2[1], e3[1]);
         }
       }
       __syncwarp();

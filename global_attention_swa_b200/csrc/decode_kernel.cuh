@@ -213,12 +213,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           l0 = l0 * a0 + ((p00 + p01) + (p10 + p11));
           l1 = l1 * a1 + ((p02 + p03) + (p12 + p13));
         }
+        // rescale O only when some row's running max moved (2^0 is exactly 1)
+        if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-          o[n][0] *= a0;
-          o[n][1] *= a0;
-          o[n][2] *= a1;
-          o[n][3] *= a1;
+          for (int n = 0; n < 16; ++n) {
+            o[n][0] *= a0;
+            o[n][1] *= a0;
+            o[n][2] *= a1;
+            o[n][3] *= a1;
+          }
         }
         // ---- O += P V.  ldmatrix.trans rows: lanes 0-7 keys kw+0..7, 8-15 keys kw+8..15
         // (dims +0), 16-23 keys kw+0..7, 24-31 keys kw+8..15 (dims +8).

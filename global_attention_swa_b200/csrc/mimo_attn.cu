@@ -183,7 +183,10 @@ DecodePlan decode_plan(int batch, int hkv, int capacity, int window) {
   pl.cap_eff = (!pl.ring && window > 0) ? std::min(window, capacity) : capacity;
   const int tile = mimo::kDecTileKeys;
   // Aim for >= 2 resident work units per SM across the grid, splits of
-  // 256..2048 keys; a single split needs no workspace and no combine.
+  // 256..16384 keys (a split's fixed costs -- query fragments, the warp merge,
+  // its partial and the combine -- fall behind its streaming from ~8K keys on:
+  // at batch 64 x 262144 slots, 16384-key splits run 9 % faster than 2048);
+  // a single split needs no workspace and no combine.
   int chunk = env_chunk();
   if (chunk <= 0) {
     const long units = (long)batch * hkv;
@@ -192,7 +195,7 @@ DecodePlan decode_plan(int batch, int hkv, int capacity, int window) {
     long max_split = std::max(1L, ((long)pl.cap_eff + 255) / 256);
     nsplit = std::max(1L, std::min(nsplit, max_split));
     long c = ((long)pl.cap_eff + nsplit - 1) / nsplit;
-    chunk = (int)std::min<long>(c, 2048);
+    chunk = (int)std::min<long>(c, 16384);
   }
   chunk = std::max(tile, ((chunk + tile - 1) / tile) * tile);
   pl.chunk = chunk;
