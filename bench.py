@@ -319,6 +319,31 @@ def run_ours(args, rank, world, peaks, peak_kind):
             "note": "e4m3 K/V caches with per-KV-head scales (the next row after the step's "
                     "kernels); not part of the step or its value"}}
         del d8
+        # decode-step rotation + append of B=64 new tokens into the 129-slot rings
+        # (latency-bound: 3.5 MB moved)
+        gq = torch.Generator(device=dev)
+        gq.manual_seed(seed + 11)
+        qn = torch.randn((64, HQ, DQK), generator=gq, device=dev).to(torch.bfloat16)
+        kn = torch.randn((64, HKV, DQK), generator=gq, device=dev).to(torch.bfloat16)
+        vn = torch.randn((64, HKV, DV), generator=gq, device=dev).to(torch.bfloat16)
+        ms_ra = []
+        for i in range(args.warmup + 20):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mimo.mimo_attn_rope_append(qn, kn, vn, dsw.k_cache, dsw.v_cache, dsw.seqlens, SWA,
+                                       10000.0)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms_ra.append(e0.elapsed_time(e1))
+        mimo.mimo_attn_device_status()
+        bytes_ra = 64 * (2 * HQ * DQK * 2 + 2 * HKV * (DQK + DV) * 2)
+        m_ra = float(np.median(ms_ra))
+        extra["rope_append_B64"] = {
+            "us": round(m_ra * 1e3, 2), "GB/s": round(bytes_ra / (m_ra * 1e-3) / 1e9, 1),
+            "algorithmic_bytes": bytes_ra, "launches": 1,
+            "note": "rotation of the new token's q (in place) and k, append of k and v to the "
+                    "129-slot rings; launch/latency-bound, L2-resident"}
 
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,

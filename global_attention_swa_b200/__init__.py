@@ -42,6 +42,7 @@ EXPORTED = (
     "mimo_attn_decode_noalloc",
     "mimo_attn_decode_fp8_workspace_size",
     "mimo_attn_decode_fp8",
+    "mimo_attn_rope_append",
 )
 
 
@@ -85,6 +86,9 @@ def _load():
     lib.mimo_attn_decode_fp8.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp,
                                          sz, vp]
     lib.mimo_attn_decode_fp8.restype = i32
+    lib.mimo_attn_rope_append.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                          ctypes.c_float, i32, vp]
+    lib.mimo_attn_rope_append.restype = i32
     return lib
 
 
@@ -195,6 +199,20 @@ def mimo_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale_kv, seqlens, wind
                                     int(window), _ptr(sinks), _ptr(out), _ptr(lse),
                                     _ptr(workspace), wbytes, _stream(stream)))
     return out, lse
+
+
+def mimo_attn_rope_append(q, k_new, v_new, k_cache, v_cache, seqlens, window, rope_theta,
+                          rotary_dim=None, stream=None):
+    """Rotate the new token's q (in place) and k, and write k, v into the cache slot of
+    position seqlens - 1 (see include/mimo_attn.h).  Returns q."""
+    B, hq, dqk = q.shape
+    C, hkv = k_cache.shape[1], k_cache.shape[2]
+    dims = make_dims(hq, hkv, dqk, v_cache.shape[3])
+    rd = dqk if rotary_dim is None else int(rotary_dim)
+    _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, C,
+                                     int(window), float(rope_theta), rd, _stream(stream)))
+    return q
 
 
 def mimo_attn_device_status(stream=None):

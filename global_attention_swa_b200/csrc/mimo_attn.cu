@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "decode_kernel.cuh"
 #include "decode_fp8_kernel.cuh"
+#include "rope_append_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
@@ -467,6 +468,47 @@ mimo_status_t mimo_attn_decode_fp8(const mimo_attn_dims_t* dims, const void* q,
                                    size_t workspace_bytes, void* stream) {
   return decode_impl(dims, q, k_cache, v_cache, true, k_scale, v_scale_kv, seqlens, batch,
                      capacity, window, sinks, out, lse, workspace, workspace_bytes, stream);
+}
+
+mimo_status_t mimo_attn_rope_append(const mimo_attn_dims_t* dims, void* q, const void* k_new,
+                                    const void* v_new, void* k_cache, void* v_cache,
+                                    const int32_t* seqlens, int batch, int capacity, int window,
+                                    float rope_theta, int rotary_dim, void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  if (window < 0) return fail(MIMO_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if (batch < 0 || capacity < 0) return fail(MIMO_ERR_INVALID_ARG, "sizes must be non-negative");
+  if (batch == 0) return ok();
+  if (capacity == 0) return fail(MIMO_ERR_INVALID_ARG, "capacity must be positive");
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta))
+    return fail(MIMO_ERR_INVALID_ARG, "rope_theta must be positive and finite");
+  if (rotary_dim < 0 || rotary_dim > dims->head_dim_qk || (rotary_dim & 1))
+    return fail(MIMO_ERR_INVALID_ARG, "rotary_dim must be even and in [0, %d] (got %d)",
+                dims->head_dim_qk, rotary_dim);
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !seqlens)
+    return fail(MIMO_ERR_INVALID_ARG, "q, k_new, v_new, caches and seqlens must be non-NULL");
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache))
+    return fail(MIMO_ERR_INVALID_ARG, "q, k_new, v_new and the caches must be 16-byte aligned");
+  if ((long)batch * capacity > 0x7fffffffL)
+    return fail(MIMO_ERR_UNSUPPORTED, "batch * capacity must fit in int32");
+  mimo::RopeAppendParams p;
+  p.q = static_cast<__nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.seqlens = seqlens;
+  p.B = batch;
+  p.C = capacity;
+  p.Hq = dims->num_heads_q;
+  p.Hkv = dims->num_heads_kv;
+  p.ring = (window > 0 && capacity == window) ? 1 : 0;
+  p.rotary_dim = rotary_dim;
+  p.theta = (double)rope_theta;
+  mimo::rope_append_kernel<<<batch, mimo::kRaThreads, 0, (cudaStream_t)stream>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "rope/append launch"))) return st;
+  return ok();
 }
 
 mimo_status_t mimo_attn_device_status(void* stream) {

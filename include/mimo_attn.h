@@ -137,6 +137,37 @@ mimo_status_t mimo_attn_decode(const mimo_attn_dims_t* dims, const void* q,
                                size_t workspace_bytes, void* stream);
 
 /*
+ * The decode step's rotation and cache write for the new token (run before
+ * mimo_attn_decode on the same stream).  MiMoV2FlashConfig.rope_parameters
+ * (rope_theta) and MiMoV2FlashModel.forward (position_ids, past_key_values);
+ * the pages fix neither theta nor the pairing, and this library takes
+ * RoFormer's rotation in the rotate-half arrangement: for i < rotary_dim/2,
+ * dimensions i and i + rotary_dim/2 turn by p * theta^(-2 i / rotary_dim) at
+ * the token's position p = seqlens[b] - 1; dimensions >= rotary_dim are left
+ * unchanged.
+ *
+ *   q          [batch, Hq, Dqk] bf16: the new token's queries, rotated IN PLACE
+ *   k_new      [batch, Hkv, Dqk] bf16: its keys before rotation
+ *   v_new      [batch, Hkv, Dv ] bf16: its values
+ *   k_cache    [batch, capacity, Hkv, Dqk] bf16: the rotated key is written
+ *              to slot p (linear) or p mod capacity (ring: window > 0 and
+ *              capacity == window); no other slot is touched
+ *   v_cache    [batch, capacity, Hkv, Dv ] bf16: the value, same slot
+ *   seqlens    [batch] int32 on the device: tokens INCLUDING the new one
+ *   rope_theta > 0; rotary_dim even, 0..Dqk (0 = no rotation, plain append)
+ *
+ * Angles are formed in double precision.  A sequence with seqlens < 1, or
+ * with p >= capacity on a linear cache, is skipped and recorded as
+ * MIMO_ERR_INVALID_ARG in the device status word.
+ */
+mimo_status_t mimo_attn_rope_append(const mimo_attn_dims_t* dims, void* q,
+                                    const void* k_new, const void* v_new,
+                                    void* k_cache, void* v_cache,
+                                    const int32_t* seqlens, int batch, int capacity,
+                                    int window, float rope_theta, int rotary_dim,
+                                    void* stream);
+
+/*
  * Workspace bytes for mimo_attn_decode_fp8 (the same split plan as the bf16
  * decode, so the same size).
  */

@@ -118,6 +118,27 @@ def test_decode_fp8_workspace_matches_bf16_plan():
     assert _decode_fp8(_dims(), batch=64, cap=262144, ws=FAKE, ws_bytes=need - 16) == mimo.MIMO_ERR_WORKSPACE
 
 
+def _rope(dims, batch=2, cap=64, window=0, theta=10000.0, rd=192, q=FAKE):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    return mimo.lib.mimo_attn_rope_append(ctypes.byref(dims), p(q), p(FAKE), p(FAKE), p(FAKE),
+                                          p(FAKE), p(FAKE), batch, cap, window, theta, rd, None)
+
+
+def test_rope_append_rejects_bad_arguments():
+    assert _rope(_dims(), theta=0.0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), theta=float("nan")) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), theta=float("inf")) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), rd=7) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), rd=194) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), rd=-2) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), window=-1) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), cap=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), q=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(), q=FAKE + 2) == mimo.MIMO_ERR_INVALID_ARG
+    assert _rope(_dims(dqk=128)) == mimo.MIMO_ERR_UNSUPPORTED
+    assert _rope(_dims(), batch=0) == mimo.MIMO_OK
+
+
 def test_last_error_is_empty_after_success():
     assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
     assert mimo.lib.mimo_attn_last_error().decode() == ""
