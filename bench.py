@@ -345,6 +345,33 @@ def run_ours(args, rank, world, peaks, peak_kind):
             "note": "rotation of the new token's q (in place) and k, append of k and v to the "
                     "129-slot rings; launch/latency-bound, L2-resident"}
 
+    # context-parallel merge of 8 parts (the gathered per-rank results of a
+    # B=64 global decode split over 8 GPUs): one launch, ~2.2 MB read
+    if extra is not None:
+        gm = torch.Generator(device=dev)
+        gm.manual_seed(seed + 13)
+        po = torch.randn((8, 64, HQ, DV), generator=gm, device=dev)
+        pl = torch.randn((8, 64, HQ), generator=gm, device=dev)
+        mo = torch.empty((64, HQ, DV), dtype=torch.bfloat16, device=dev)
+        ml = torch.empty((64, HQ), dtype=torch.float32, device=dev)
+        ms_m = []
+        for i in range(args.warmup + 20):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mimo.mimo_attn_decode_merge(po, pl, dsw.sinks, out=mo, lse=ml)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms_m.append(e0.elapsed_time(e1))
+        mimo.mimo_attn_device_status()
+        bytes_m = po.numel() * 4 + pl.numel() * 4 + mo.numel() * 2 + ml.numel() * 4
+        m_m = float(np.median(ms_m))
+        extra["decode_merge_R8_B64"] = {
+            "us": round(m_m * 1e3, 2), "GB/s": round(bytes_m / (m_m * 1e-3) / 1e9, 1),
+            "algorithmic_bytes": bytes_m, "launches": 1,
+            "note": "log-sum-exp merge of 8 context-parallel parts with the sink; the all-gather "
+                    "before it is NCCL (not run on one GPU)"}
+
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),

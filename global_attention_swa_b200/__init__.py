@@ -43,6 +43,7 @@ EXPORTED = (
     "mimo_attn_decode_fp8_workspace_size",
     "mimo_attn_decode_fp8",
     "mimo_attn_rope_append",
+    "mimo_attn_decode_merge",
 )
 
 
@@ -89,6 +90,8 @@ def _load():
     lib.mimo_attn_rope_append.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                           ctypes.c_float, i32, vp]
     lib.mimo_attn_rope_append.restype = i32
+    lib.mimo_attn_decode_merge.argtypes = [dp, vp, vp, i32, i32, vp, vp, vp, vp]
+    lib.mimo_attn_decode_merge.restype = i32
     return lib
 
 
@@ -213,6 +216,21 @@ def mimo_attn_rope_append(q, k_new, v_new, k_cache, v_cache, seqlens, window, ro
                                      _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, C,
                                      int(window), float(rope_theta), rd, _stream(stream)))
     return q
+
+
+def mimo_attn_decode_merge(part_out, part_lse, sinks, out=None, lse=None,
+                           out_dtype=torch.bfloat16, v_scale=1.0, return_lse=True, stream=None):
+    """Merge per-part decode results (part_out [R,B,Hq,128] fp32, part_lse [R,B,Hq] fp32)
+    with the sink.  Returns (out [B,Hq,128], lse [B,Hq] or None)."""
+    R, B, hq, dv = part_out.shape
+    if out is None:
+        out = torch.empty((B, hq, dv), dtype=out_dtype, device=part_out.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=part_out.device)
+    dims = make_dims(hq, 1, 192, dv, None, v_scale, out.dtype)
+    _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out), _ptr(part_lse), R, B,
+                                      _ptr(sinks), _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def mimo_attn_device_status(stream=None):

@@ -15,6 +15,7 @@
 #include "decode_kernel.cuh"
 #include "decode_fp8_kernel.cuh"
 #include "rope_append_kernel.cuh"
+#include "decode_merge_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
@@ -508,6 +509,38 @@ mimo_status_t mimo_attn_rope_append(const mimo_attn_dims_t* dims, void* q, const
   p.theta = (double)rope_theta;
   mimo::rope_append_kernel<<<batch, mimo::kRaThreads, 0, (cudaStream_t)stream>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "rope/append launch"))) return st;
+  return ok();
+}
+
+mimo_status_t mimo_attn_decode_merge(const mimo_attn_dims_t* dims, const float* part_out,
+                                     const float* part_lse, int num_parts, int batch,
+                                     const float* sinks, void* out, float* lse, void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  if (num_parts < 1) return fail(MIMO_ERR_INVALID_ARG, "num_parts must be >= 1 (got %d)", num_parts);
+  if (batch < 0) return fail(MIMO_ERR_INVALID_ARG, "batch must be non-negative");
+  if (batch == 0) return ok();
+  if (!part_out || !part_lse || !out)
+    return fail(MIMO_ERR_INVALID_ARG, "part_out, part_lse and out must be non-NULL");
+  if (!aligned16(part_out) || !aligned16(out) || ((uintptr_t)part_lse & 3u) ||
+      (lse && ((uintptr_t)lse & 3u)) || (sinks && ((uintptr_t)sinks & 3u)))
+    return fail(MIMO_ERR_INVALID_ARG, "part_out and out must be 16-byte aligned");
+  const long warps = (long)batch * dims->num_heads_q;
+  if (warps * 32 > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "batch * Hq too large");
+  mimo::DecodeMergeParams p;
+  p.part_out = part_out;
+  p.part_lse = part_lse;
+  p.sinks = sinks;
+  p.out = out;
+  p.lse = lse;
+  p.R = num_parts;
+  p.B = batch;
+  p.Hq = dims->num_heads_q;
+  p.v_scale = v_scale_of(dims);
+  p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+  const int blocks = (int)((warps * 32 + 255) / 256);
+  mimo::decode_merge_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "decode merge launch"))) return st;
   return ok();
 }
 

@@ -168,6 +168,30 @@ mimo_status_t mimo_attn_rope_append(const mimo_attn_dims_t* dims, void* q,
                                     void* stream);
 
 /*
+ * Merge of decode results over disjoint parts of each sequence's keys
+ * (context parallelism: a global layer's cache split across GPUs, each part
+ * decoded with mimo_attn_decode, window 0, sinks = NULL, fp32 out and lse,
+ * then gathered).  MiMo-V2-Flash model doc, "Key features" (learnable sink):
+ *
+ *   M   = max(sigma_h, max_r lse_r)
+ *   Z   = exp(sigma_h - M) + sum_r exp(lse_r - M)
+ *   out = dims->v_scale * sum_r exp(lse_r - M) out_r / Z,   lse = M + ln Z
+ *
+ *   part_out [num_parts, batch, Hq, Dv] fp32 (16-byte aligned)
+ *   part_lse [num_parts, batch, Hq] fp32, natural log; -inf marks a part
+ *            with no keys for that sequence (its part_out is then ignored)
+ *   sinks    [Hq] fp32 or NULL;  out [batch, Hq, Dv] in dims->out_dtype;
+ *   lse      [batch, Hq] fp32 or NULL
+ *
+ * The parts' order does not matter.  With every part empty and no sink the
+ * output is 0 and lse -inf.
+ */
+mimo_status_t mimo_attn_decode_merge(const mimo_attn_dims_t* dims, const float* part_out,
+                                     const float* part_lse, int num_parts, int batch,
+                                     const float* sinks, void* out, float* lse,
+                                     void* stream);
+
+/*
  * Workspace bytes for mimo_attn_decode_fp8 (the same split plan as the bf16
  * decode, so the same size).
  */

@@ -12,6 +12,9 @@ Modules
 -------
 ``attention``  vectorised fp64 prefill and decode (NumPy matmuls per query block).
 ``brute``      scalar triple loops for tiny shapes, used to pin ``attention``.
+``merge``      merging decode results over disjoint parts of a cache (context
+               parallelism) with the sink.
+``rope``       rotary embedding and the decode-step cache append.
 ``fp8``        e4m3 decoding from the format's definition and decode over FP8
                KV caches with per-KV-head scales (``attention.decode`` on the
                dequantised caches).

@@ -139,6 +139,17 @@ def test_rope_append_rejects_bad_arguments():
     assert _rope(_dims(), batch=0) == mimo.MIMO_OK
 
 
+def test_decode_merge_rejects_bad_arguments():
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    call = lambda nparts=2, batch=2, po=FAKE, out=FAKE: mimo.lib.mimo_attn_decode_merge(  # noqa: E731
+        ctypes.byref(_dims()), p(po), p(FAKE), nparts, batch, None, p(out), None, None)
+    assert call(nparts=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert call(batch=-1) == mimo.MIMO_ERR_INVALID_ARG
+    assert call(po=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert call(out=FAKE + 8) == mimo.MIMO_ERR_INVALID_ARG
+    assert call(batch=0) == mimo.MIMO_OK
+
+
 def test_last_error_is_empty_after_success():
     assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
     assert mimo.lib.mimo_attn_last_error().decode() == ""
