@@ -506,8 +506,14 @@ mimo_status_t mimo_attn_rope_append(const mimo_attn_dims_t* dims, void* q, const
   p.Hkv = dims->num_heads_kv;
   p.ring = (window > 0 && capacity == window) ? 1 : 0;
   p.rotary_dim = rotary_dim;
-  p.theta = (double)rope_theta;
-  mimo::rope_append_kernel<<<batch, mimo::kRaThreads, 0, (cudaStream_t)stream>>>(p);
+  for (int i = 0; i < mimo::kRaMaxHalf; ++i)
+    p.inv_freq[i] = (rotary_dim > 0 && i < rotary_dim / 2)
+                        ? std::pow((double)rope_theta, -2.0 * i / (double)rotary_dim)
+                        : 0.0;
+  if (batch > 0x7fffffff || p.Hq > 65535 * mimo::kRaHeadsPerCta)
+    return fail(MIMO_ERR_UNSUPPORTED, "batch or Hq too large");
+  const dim3 grid(batch, (p.Hq + mimo::kRaHeadsPerCta - 1) / mimo::kRaHeadsPerCta + 1);
+  mimo::rope_append_kernel<<<grid, mimo::kRaThreads, 0, (cudaStream_t)stream>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "rope/append launch"))) return st;
   return ok();
 }

@@ -52,7 +52,7 @@ def _run(lengths, cap, window, theta, rotary_dim, seed):
     (129, 129, [1, 128, 129, 130, 1000]),     # ring: wraps past the capacity
     (129, 4096, [1, 200, 4096]),              # linear cache with a window
 ])
-@pytest.mark.parametrize("theta,rotary_dim", [(10000.0, 192), (1.0e6, 64)])
+@pytest.mark.parametrize("theta,rotary_dim", [(10000.0, 192), (1.0e6, 64), (500.0, 60)])
 def test_rotation_and_append_match_oracle(window, cap, lengths, theta, rotary_dim):
     x, qd, kc, vc, rq, rk, rv = _run(lengths, cap, window, theta, rotary_dim, seed=cap + window)
     _close(qd, rq, "q")
