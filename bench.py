@@ -391,6 +391,37 @@ def run_ours(args, rank, world, peaks, peak_kind):
                     "time per call (CUDA graph replay); the all-gather before it is NCCL (not run "
                     "on one GPU)"}
 
+    # prefill backward of one global layer at T=8192 (training; row next-3)
+    if extra is not None:
+        Tb = 8192
+        xb = W.prefill_inputs([Tb], seed=seed + 17, device=dev)
+        ob, lb = mimo.mimo_attn_prefill(xb.q, xb.k, xb.v, xb.sinks, 0, xb.cu_seqlens, Tb)
+        gb = torch.Generator(device=dev)
+        gb.manual_seed(seed + 19)
+        dob = torch.randn(ob.shape, generator=gb, device=dev).to(ob.dtype)
+        ms_b = []
+        for i in range(args.warmup + 5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            mimo.mimo_attn_prefill_backward(xb.q, xb.k, xb.v, ob, lb, dob, xb.sinks, 0,
+                                            xb.cu_seqlens, Tb)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms_b.append(e0.elapsed_time(e1))
+        mimo.mimo_attn_device_status()
+        pairs = Tb * (Tb + 1) // 2
+        fb = 1664 * HQ * pairs  # S, dP, dV, dK, dQ: 2 x (192 + 128 + 128 + 192 + 192) per pair and head
+        m_b = float(np.mean(ms_b))
+        extra["prefill_backward_global_T8192"] = {
+            "ms": round(m_b, 3), "TFLOP/s": round(fb / (m_b * 1e-3) / 1e12, 1),
+            "roofline_frac": round(fb / (m_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "bound": "tensor", "useful_flop": fb, "launches": 5,
+            "note": "dq, dk, dv, dsinks with warp-level mma.sync (the forward's out and lse as "
+                    "inputs); the dV pass recomputes S"}
+        del xb, ob, lb, dob
+
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),

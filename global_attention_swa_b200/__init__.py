@@ -44,6 +44,8 @@ EXPORTED = (
     "mimo_attn_decode_fp8",
     "mimo_attn_rope_append",
     "mimo_attn_decode_merge",
+    "mimo_attn_prefill_backward_workspace_size",
+    "mimo_attn_prefill_backward",
 )
 
 
@@ -92,6 +94,11 @@ def _load():
     lib.mimo_attn_rope_append.restype = i32
     lib.mimo_attn_decode_merge.argtypes = [dp, vp, vp, i32, i32, vp, vp, vp, vp]
     lib.mimo_attn_decode_merge.restype = i32
+    lib.mimo_attn_prefill_backward_workspace_size.argtypes = [dp, i32]
+    lib.mimo_attn_prefill_backward_workspace_size.restype = sz
+    lib.mimo_attn_prefill_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
+                                               vp, vp, vp, vp, vp, sz, vp]
+    lib.mimo_attn_prefill_backward.restype = i32
     return lib
 
 
@@ -231,6 +238,29 @@ def mimo_attn_decode_merge(part_out, part_lse, sinks, out=None, lse=None,
     _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out), _ptr(part_lse), R, B,
                                       _ptr(sinks), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def mimo_attn_prefill_backward(q, k, v, out, lse, dout, sinks, window, cu_seqlens, max_seqlen,
+                               softmax_scale=None, v_scale=1.0, stream=None):
+    """Gradients of mimo_attn_prefill: returns (dq, dk, dv [fp32], dsinks [Hq] fp32 or None).
+
+    ``out`` and ``lse`` are the forward's results; ``dout`` has out's dtype.
+    """
+    nt, hq, dqk = q.shape
+    hkv, dv_dim = k.shape[1], v.shape[2]
+    dq = torch.empty((nt, hq, dqk), dtype=torch.float32, device=q.device)
+    dk = torch.empty((nt, hkv, dqk), dtype=torch.float32, device=q.device)
+    dv = torch.empty((nt, hkv, dv_dim), dtype=torch.float32, device=q.device)
+    ds = None if sinks is None else torch.empty(hq, dtype=torch.float32, device=q.device)
+    dims = make_dims(hq, hkv, dqk, dv_dim, softmax_scale, v_scale, out.dtype)
+    need = int(lib.mimo_attn_prefill_backward_workspace_size(ctypes.byref(dims), nt))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib.mimo_attn_prefill_backward(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                          _ptr(lse), _ptr(dout), _ptr(sinks), int(window),
+                                          _ptr(cu_seqlens), cu_seqlens.numel() - 1, nt,
+                                          int(max_seqlen), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds),
+                                          _ptr(ws), ws.numel(), _stream(stream)))
+    return dq, dk, dv, ds
 
 
 def mimo_attn_device_status(stream=None):

@@ -16,6 +16,7 @@
 #include "decode_fp8_kernel.cuh"
 #include "rope_append_kernel.cuh"
 #include "decode_merge_kernel.cuh"
+#include "backward_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
@@ -140,6 +141,21 @@ mimo_status_t ensure_attributes() {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kDecSmemBytes),
                        "decode smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dq_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kBwSmemBytes),
+                       "backward dq smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kBwSmemBytes),
+                       "backward dv smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_kernel<false>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kBwSmemBytes),
+                       "backward dk smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_fp8_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -547,6 +563,87 @@ mimo_status_t mimo_attn_decode_merge(const mimo_attn_dims_t* dims, const float* 
   const int blocks = (int)((warps * 32 + 255) / 256);
   mimo::decode_merge_kernel<<<blocks, 256, 0, (cudaStream_t)stream>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "decode merge launch"))) return st;
+  return ok();
+}
+
+size_t mimo_attn_prefill_backward_workspace_size(const mimo_attn_dims_t* dims, int total_tokens) {
+  if (!dims || dims->num_heads_q <= 0 || total_tokens <= 0) return 0;
+  return (size_t)2 * dims->num_heads_q * total_tokens * sizeof(float);
+}
+
+mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const void* q, const void* k,
+                                         const void* v, const void* out, const float* lse,
+                                         const void* dout, const float* sinks, int window,
+                                         const int32_t* cu_seqlens, int num_seqs,
+                                         int total_tokens, int max_seqlen, float* dq, float* dk,
+                                         float* dv, float* dsinks, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  mimo_status_t st = check_dims(dims);
+  if (st) return st;
+  if (window < 0) return fail(MIMO_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0)
+    return fail(MIMO_ERR_INVALID_ARG, "sizes must be non-negative");
+  if (!cu_seqlens) return fail(MIMO_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (total_tokens == 0 || num_seqs == 0 || max_seqlen == 0) return ok();
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv)
+    return fail(MIMO_ERR_INVALID_ARG, "q, k, v, out, lse, dout, dq, dk and dv must be non-NULL");
+  if (sinks && !dsinks) return fail(MIMO_ERR_INVALID_ARG, "dsinks is NULL while sinks is given");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || ((uintptr_t)lse & 3u) ||
+      (sinks && ((uintptr_t)sinks & 3u)) || (dsinks && ((uintptr_t)dsinks & 3u)))
+    return fail(MIMO_ERR_INVALID_ARG, "tensors must be 16-byte aligned (lse, sinks, dsinks 4-byte)");
+  if (max_seqlen > total_tokens)
+    return fail(MIMO_ERR_INVALID_ARG, "max_seqlen (%d) exceeds total_tokens (%d)", max_seqlen,
+                total_tokens);
+  if (num_seqs > 65535) return fail(MIMO_ERR_UNSUPPORTED, "num_seqs > 65535");
+  const size_t need = mimo_attn_prefill_backward_workspace_size(dims, total_tokens);
+  if (!workspace || workspace_bytes < need)
+    return fail(MIMO_ERR_WORKSPACE, "backward workspace of %zu bytes needed (got %zu)", need,
+                workspace_bytes);
+  if ((uintptr_t)workspace & 15u) return fail(MIMO_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((long)total_tokens * dims->num_heads_q * 32 > 0x7fffffffL * 255L)
+    return fail(MIMO_ERR_UNSUPPORTED, "total_tokens * Hq too large");
+  if ((st = ensure_attributes())) return st;
+  mimo::BackwardParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.out = out;
+  p.dout = dout;
+  p.lse = lse;
+  p.sinks = sinks;
+  p.cu_seqlens = cu_seqlens;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dsinks = dsinks;
+  p.D = static_cast<float*>(workspace);
+  p.psd = p.D + (size_t)dims->num_heads_q * total_tokens;
+  p.total = total_tokens;
+  p.Hq = dims->num_heads_q;
+  p.Hkv = dims->num_heads_kv;
+  p.G = p.Hq / p.Hkv;
+  p.window = window;
+  p.num_seqs = num_seqs;
+  p.scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / std::sqrt((float)dims->head_dim_qk);
+  p.scale_log2 = scale_log2_of(dims);
+  p.v_scale = v_scale_of(dims);
+  p.io_f32 = dims->out_dtype == MIMO_DTYPE_F32;
+  cudaStream_t s = (cudaStream_t)stream;
+  const long pre_threads = (long)total_tokens * p.Hq * 32;
+  mimo::bwd_preprocess_kernel<<<(unsigned)((pre_threads + 255) / 256), 256, 0, s>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "backward preprocess launch"))) return st;
+  if (sinks) {
+    mimo::bwd_sink_kernel<<<p.Hq, 256, 0, s>>>(p);
+    if ((st = cuda_check(cudaGetLastError(), "backward sink launch"))) return st;
+  }
+  const int tiles = (max_seqlen + mimo::kBwTile - 1) / mimo::kBwTile;
+  mimo::bwd_dq_kernel<<<dim3(tiles, p.Hq, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "backward dq launch"))) return st;
+  mimo::bwd_dkv_kernel<true><<<dim3(tiles, p.Hkv, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "backward dv launch"))) return st;
+  mimo::bwd_dkv_kernel<false><<<dim3(tiles, p.Hkv, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  if ((st = cuda_check(cudaGetLastError(), "backward dk launch"))) return st;
   return ok();
 }
 

@@ -192,6 +192,44 @@ mimo_status_t mimo_attn_decode_merge(const mimo_attn_dims_t* dims, const float* 
                                      void* stream);
 
 /*
+ * Workspace bytes for mimo_attn_prefill_backward: 2 * Hq * total_tokens fp32.
+ */
+size_t mimo_attn_prefill_backward_workspace_size(const mimo_attn_dims_t* dims,
+                                                 int total_tokens);
+
+/*
+ * Gradients of mimo_attn_prefill (training).  MiMo-V2-Flash model doc, "Key
+ * features": the attention-sink bias is learnable, so it has a gradient.
+ * Per query head h, row i, visible key j (S = s <q_i, k_j>, P = exp(S - lse_i)):
+ *   D_i = <dO_i, O_i>;  dS_ij = P_ij (v_scale <dO_i, v_j> - D_i)
+ *   dq_i = s sum_j dS_ij k_j;  dk_j = s sum dS_ij q_i;  dv_j = v_scale sum P_ij dO_i
+ *   (dk, dv summed over the query heads of j's key/value head)
+ *   dsinks_h = -sum_i exp(sinks_h - lse_i) D_i
+ *
+ *   q, k, v, sinks, window, cu_seqlens, num_seqs, total_tokens, max_seqlen:
+ *              as passed to mimo_attn_prefill
+ *   out, lse   the forward's out (dims->out_dtype) and lse [Hq, total_tokens]
+ *   dout       [total_tokens, Hq, Dv], same dtype as out
+ *   dq         [total_tokens, Hq,  Dqk] fp32;  dk [total_tokens, Hkv, Dqk] fp32
+ *   dv         [total_tokens, Hkv, Dv ] fp32 (all three overwritten)
+ *   dsinks     [Hq] fp32, required when sinks is given (ignored otherwise)
+ *   workspace  >= mimo_attn_prefill_backward_workspace_size() bytes, 16-byte aligned
+ *
+ * Warp-level tensor-core kernels (mma.sync, bf16 operands, fp32
+ * accumulation; P and dS rounded to bf16 as operands); deterministic: no
+ * atomics.
+ */
+mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const void* q,
+                                         const void* k, const void* v, const void* out,
+                                         const float* lse, const void* dout,
+                                         const float* sinks, int window,
+                                         const int32_t* cu_seqlens, int num_seqs,
+                                         int total_tokens, int max_seqlen, float* dq,
+                                         float* dk, float* dv, float* dsinks,
+                                         void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
  * Workspace bytes for mimo_attn_decode_fp8 (the same split plan as the bf16
  * decode, so the same size).
  */

@@ -150,6 +150,27 @@ def test_decode_merge_rejects_bad_arguments():
     assert call(batch=0) == mimo.MIMO_OK
 
 
+def _bwd(dims, sinks=None, dsinks=None, ws=FAKE, ws_bytes=1 << 30, total=128, maxlen=128, dq=FAKE):
+    p = lambda x: ctypes.c_void_p(x) if x else None  # noqa: E731
+    return mimo.lib.mimo_attn_prefill_backward(
+        ctypes.byref(dims), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(FAKE), p(sinks), 0,
+        p(FAKE), 1, total, maxlen, p(dq), p(FAKE), p(FAKE), p(dsinks), p(ws), ws_bytes, None)
+
+
+def test_prefill_backward_rejects_bad_arguments():
+    need = mimo.lib.mimo_attn_prefill_backward_workspace_size(ctypes.byref(_dims()), 128)
+    assert need == 2 * 64 * 128 * 4
+    assert _bwd(_dims(), sinks=FAKE, dsinks=None) == mimo.MIMO_ERR_INVALID_ARG
+    assert "dsinks" in mimo.lib.mimo_attn_last_error().decode()
+    assert _bwd(_dims(), ws=None) == mimo.MIMO_ERR_WORKSPACE
+    assert _bwd(_dims(), ws_bytes=need - 4) == mimo.MIMO_ERR_WORKSPACE
+    assert _bwd(_dims(), dq=0) == mimo.MIMO_ERR_INVALID_ARG
+    assert _bwd(_dims(), dq=FAKE + 4) == mimo.MIMO_ERR_INVALID_ARG
+    assert _bwd(_dims(), maxlen=129) == mimo.MIMO_ERR_INVALID_ARG
+    assert _bwd(_dims(dv=192)) == mimo.MIMO_ERR_UNSUPPORTED
+    assert _bwd(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
+
+
 def test_last_error_is_empty_after_success():
     assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
     assert mimo.lib.mimo_attn_last_error().decode() == ""

@@ -1,0 +1,79 @@
+"""Prefill backward (mimo_attn_prefill_backward) vs the fp64 oracle backward.
+
+The forward runs on the GPU (its out and lse feed the backward, as in
+training); the oracle recomputes everything in fp64.  Tolerance per gradient
+tensor: relative Frobenius error <= 1e-2 and every element within
+1e-2 * max|ref| + 1e-4 -- the kernels round P and dS to bf16 as MMA operands
+(2^-8 relative each), like P in the forward, and accumulate in fp32; the
+1e-4 floor covers gradients that are exactly zero in exact arithmetic (a row
+with one visible key and no sink: D and dP cancel up to fp32 summation order),
+next to gradient magnitudes of 0.1-10 here.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle.backward import prefill_backward
+from tests import parity_util as P
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import global_attention_swa_b200 as mimo
+
+
+def grad_check(got, ref, what):
+    g = P.to64(got)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite"
+    scale = np.abs(ref).max()
+    err = np.abs(g - ref)
+    assert err.max() <= 1e-2 * scale + 1e-4, f"{what}: max err {err.max():.3e} vs scale {scale:.3e}"
+    if scale > 1e-3:
+        fro = np.linalg.norm(g - ref) / np.linalg.norm(ref)
+        assert fro <= 1e-2, f"{what}: rel-Frobenius {fro:.3e}"
+    else:
+        fro = 0.0
+    return fro
+
+
+def _run(lengths, hq, hkv, window, sinks, out_dtype, seed, v_scale=1.0):
+    x = W.prefill_inputs(lengths, hq=hq, hkv=hkv, seed=seed, sinks=sinks, device="cuda")
+    maxlen = max(lengths)
+    out, lse = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, maxlen,
+                                      out_dtype=out_dtype, v_scale=v_scale)
+    g = torch.Generator(device="cuda").manual_seed(seed + 1)
+    dout = torch.randn(out.shape, generator=g, device="cuda").to(out_dtype)
+    dq, dk, dv, ds = mimo.mimo_attn_prefill_backward(x.q, x.k, x.v, out, lse, dout, x.sinks, window,
+                                                     x.cu_seqlens, maxlen, v_scale=v_scale)
+    mimo.mimo_attn_device_status()
+    rq, rk, rv, rs = prefill_backward(x.q, x.k, x.v, dout, x.sinks, window, x.cu_seqlens,
+                                      v_scale=v_scale)
+    return (dq, dk, dv, ds), (rq, rk, rv, rs)
+
+
+@pytest.mark.parametrize("window", [129, 0, 1])
+@pytest.mark.parametrize("sinks", [True, False])
+def test_tiny_heads(window, sinks):
+    got, ref = _run([512], 16, 1, window, sinks, torch.float32, seed=window + 3)
+    for name, a, b in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
+        grad_check(a, b, f"{name} W={window}")
+    if sinks:
+        grad_check(got[3], ref[3], "dsinks")
+    else:
+        assert got[3] is None
+
+
+@pytest.mark.parametrize("window", [129, 0])
+def test_model_heads_varlen_bf16(window):
+    got, ref = _run([300, 0, 129, 64, 1], 64, 4, window, True, torch.bfloat16, seed=11, v_scale=0.707)
+    for name, a, b in zip(("dq", "dk", "dv", "dsinks"), got, ref):
+        grad_check(a, b, f"{name} W={window}")
+
+
+def test_deterministic():
+    a, _ = _run([200, 70], 16, 2, 129, True, torch.float32, seed=5)
+    b, _ = _run([200, 70], 16, 2, 129, True, torch.float32, seed=5)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

@@ -1,0 +1,74 @@
+"""Pins for the oracle's attention backward, against central finite differences
+of the forward oracle (CPU only).
+
+Loss = sum(out * W) for a fixed random W, so dO = W; every element of q, k, v
+and the sink logits is perturbed by +-h and the loss difference compared with
+the analytic gradient.  A backward that dropped the sink's gradient, the
+D = <dO, O> term or the GQA sum over heads fails these.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.backward import prefill_backward
+
+
+def _loss(q, k, v, s, W, window, cu, scale, v_scale):
+    out, _ = oracle.prefill(q, k, v, s, window, cu, scale=scale, v_scale=v_scale)
+    return float((out * W).sum())
+
+
+def _fd(f, x, h=1e-6):
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + h
+        fp = f()
+        x[i] = old - h
+        fm = f()
+        x[i] = old
+        g[i] = (fp - fm) / (2 * h)
+    return g
+
+
+@pytest.mark.parametrize("window,lengths", [(0, [7]), (3, [7]), (0, [3, 0, 5]), (2, [4, 6])])
+@pytest.mark.parametrize("sinks", [True, False])
+def test_gradients_match_finite_differences(window, lengths, sinks):
+    rng = np.random.default_rng(sum(lengths) + window)
+    Nt = sum(lengths)
+    Hq, Hkv, Dqk, Dv = 4, 2, 5, 3
+    q = rng.standard_normal((Nt, Hq, Dqk))
+    k = rng.standard_normal((Nt, Hkv, Dqk))
+    v = rng.standard_normal((Nt, Hkv, Dv))
+    s = rng.standard_normal(Hq) if sinks else None
+    W = rng.standard_normal((Nt, Hq, Dv))
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    scale, v_scale = 0.37, 0.8
+    f = lambda: _loss(q, k, v, s, W, window, cu, scale, v_scale)  # noqa: E731
+    dq, dk, dv, ds = prefill_backward(q, k, v, W, s, window, cu, scale=scale, v_scale=v_scale)
+    np.testing.assert_allclose(dq, _fd(f, q), atol=2e-8)
+    np.testing.assert_allclose(dk, _fd(f, k), atol=2e-8)
+    np.testing.assert_allclose(dv, _fd(f, v), atol=2e-8)
+    if sinks:
+        np.testing.assert_allclose(ds, _fd(f, s), atol=2e-8)
+    else:
+        assert ds is None
+
+
+def test_pins_have_teeth():
+    """Dropping the sink gradient or the D term changes the result."""
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((6, 2, 4))
+    k = rng.standard_normal((6, 1, 4))
+    v = rng.standard_normal((6, 1, 3))
+    s = np.array([1.5, -0.5])
+    W = rng.standard_normal((6, 2, 3))
+    cu = np.array([0, 6])
+    dq, dk, dv, ds = prefill_backward(q, k, v, W, s, 0, cu)
+    assert np.abs(ds).max() > 1e-3                     # the sink has a real gradient
+    out, _ = oracle.prefill(q, k, v, s, 0, cu)
+    D = (W * out).sum(axis=2)
+    assert np.abs(D).max() > 1e-3                      # D matters for dS
