@@ -144,17 +144,17 @@ mimo_status_t ensure_attributes() {
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dq_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            mimo::kBwSmemBytes),
+                                            mimo::kBqSmemBytes),
                        "backward dq smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_kernel<true>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            mimo::kBwSmemBytes),
+                                            mimo::kBkSmemBytes),
                        "backward dv smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_kernel<false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            mimo::kBwSmemBytes),
+                                            mimo::kBkSmemBytes),
                        "backward dk smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_fp8_kernel,
@@ -638,11 +638,13 @@ mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const voi
     if ((st = cuda_check(cudaGetLastError(), "backward sink launch"))) return st;
   }
   const int tiles = (max_seqlen + mimo::kBwTile - 1) / mimo::kBwTile;
-  mimo::bwd_dq_kernel<<<dim3(tiles, p.Hq, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  const int qtiles = (max_seqlen + mimo::kBqRows - 1) / mimo::kBqRows;
+  mimo::bwd_dq_kernel<<<dim3(qtiles, p.Hq, num_seqs), mimo::kBkThreads, mimo::kBqSmemBytes, s>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "backward dq launch"))) return st;
-  mimo::bwd_dkv_kernel<true><<<dim3(tiles, p.Hkv, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  const dim3 kv_grid((unsigned)tiles * p.Hkv, num_seqs);  // (key tile, KV head) per CTA
+  mimo::bwd_dkv_kernel<true><<<kv_grid, mimo::kBkThreads, mimo::kBkSmemBytes, s>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "backward dv launch"))) return st;
-  mimo::bwd_dkv_kernel<false><<<dim3(tiles, p.Hkv, num_seqs), mimo::kBwThreads, mimo::kBwSmemBytes, s>>>(p);
+  mimo::bwd_dkv_kernel<false><<<kv_grid, mimo::kBkThreads, mimo::kBkSmemBytes, s>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "backward dk launch"))) return st;
   return ok();
 }
