@@ -18,6 +18,10 @@ Modules
 ``fp8``        e4m3 decoding from the format's definition and decode over FP8
                KV caches with per-KV-head scales (``attention.decode`` on the
                dequantised caches).
+``backward``   gradients of the prefill (q, k, v and the sink logits) from
+               explicit probability matrices, pinned to finite differences;
+               ``prefill_backward_sampled`` gives them at chosen positions of
+               one long sequence.
 
 Every function here is pinned by a ``-m "not gpu"`` test against something
 other than itself (brute force, closed forms, a library special case, or the

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import workloads as W
-from oracle.backward import prefill_backward
+from oracle.backward import prefill_backward, prefill_backward_sampled
 from tests import parity_util as P
 
 pytestmark = pytest.mark.gpu
@@ -77,3 +77,43 @@ def test_deterministic():
     b, _ = _run([200, 70], 16, 2, 129, True, torch.float32, seed=5)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def sampled_check(got, ref, what):
+    """Per-element bound of grad_check over a sample (scale = the sample's max |ref|)."""
+    g = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite"
+    scale = np.abs(ref).max()
+    err = np.abs(g - ref).max()
+    assert err <= 1e-2 * scale + 1e-4, f"{what}: max err {err:.3e} vs scale {scale:.3e}"
+    fro = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert fro <= 1e-2, f"{what}: rel-Frobenius {fro:.3e}"
+
+
+@pytest.mark.parametrize("T,window,q_rows,k_rows", [
+    # the benchmark's backward: one global layer at T=8192 (keys near the end: the
+    # oracle needs every query row that sees a key)
+    (8192, 0, [0, 1, 63, 64, 127, 128, 4095, 4096, 8190, 8191], [7690, 8000, 8127, 8128, 8191]),
+    # a sliding-window layer at T=32768, keys anywhere
+    (32768, 129, [0, 128, 129, 16383, 32767], [0, 1, 63, 64, 20000, 32640, 32767]),
+])
+def test_full_size_sampled(T, window, q_rows, k_rows):
+    """Model head shape, bf16 forward output, full length, in the launch configuration the
+    benchmark times; the oracle gives dq, dk, dv and dsinks at sampled positions."""
+    x = W.prefill_inputs([T], seed=T + window, device="cuda")
+    out, lse = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, T)
+    g = torch.Generator(device="cuda").manual_seed(T + window + 1)
+    dout = torch.randn(out.shape, generator=g, device="cuda").to(out.dtype)
+    dq, dk, dv, ds = mimo.mimo_attn_prefill_backward(x.q, x.k, x.v, out, lse, dout, x.sinks, window,
+                                                     x.cu_seqlens, T)
+    mimo.mimo_attn_device_status()
+    q_heads, kv_heads, sink_heads = [0, 17, 63], [0, 3], [5, 60]
+    rq, rk, rv, rs = prefill_backward_sampled(x.q.cpu(), x.k.cpu(), x.v.cpu(), dout.cpu(), x.sinks.cpu(),
+                                              window, q_rows, q_heads, k_rows, kv_heads,
+                                              sink_heads=sink_heads)
+    sampled_check(dq[q_rows][:, q_heads].cpu(), rq, f"dq T={T}")
+    sampled_check(dk[k_rows][:, kv_heads].cpu(), rk, f"dk T={T}")
+    sampled_check(dv[k_rows][:, kv_heads].cpu(), rv, f"dv T={T}")
+    sampled_check(ds[sink_heads].cpu(), rs, f"dsinks T={T}")
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())

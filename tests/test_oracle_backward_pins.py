@@ -72,3 +72,50 @@ def test_pins_have_teeth():
     out, _ = oracle.prefill(q, k, v, s, 0, cu)
     D = (W * out).sum(axis=2)
     assert np.abs(D).max() > 1e-3                      # D matters for dS
+
+
+@pytest.mark.parametrize("window", [0, 3])
+@pytest.mark.parametrize("sinks", [True, False])
+def test_sampled_gradients_match_finite_differences(window, sinks):
+    """The sampled-position backward (used at sizes the full one cannot reach)
+    against central differences of the forward, with blocks smaller than the
+    sequence so that its row blocking is exercised."""
+    rng = np.random.default_rng(40 + window)
+    n, Hq, Hkv, Dqk, Dv = 9, 4, 2, 5, 3
+    q = rng.standard_normal((n, Hq, Dqk))
+    k = rng.standard_normal((n, Hkv, Dqk))
+    v = rng.standard_normal((n, Hkv, Dv))
+    s = rng.standard_normal(Hq) if sinks else None
+    W = rng.standard_normal((n, Hq, Dv))
+    cu = np.array([0, n])
+    scale, v_scale = 0.41, 1.3
+    f = lambda: _loss(q, k, v, s, W, window, cu, scale, v_scale)  # noqa: E731
+    gq, gk, gv = _fd(f, q), _fd(f, k), _fd(f, v)
+    q_rows, q_heads, k_rows, kv_heads = [0, 4, 8], [1, 3], [0, 5, 8], [0, 1]
+    dq, dk, dv, ds = oracle.backward.prefill_backward_sampled(
+        q, k, v, W, s, window, q_rows, q_heads, k_rows, kv_heads, sink_heads=[0, 2] if sinks else (),
+        scale=scale, v_scale=v_scale, block=4)
+    np.testing.assert_allclose(dq, gq[np.ix_(q_rows, q_heads)], atol=2e-8)
+    np.testing.assert_allclose(dk, gk[np.ix_(k_rows, kv_heads)], atol=2e-8)
+    np.testing.assert_allclose(dv, gv[np.ix_(k_rows, kv_heads)], atol=2e-8)
+    if sinks:
+        np.testing.assert_allclose(ds, _fd(f, s)[[0, 2]], atol=2e-8)
+
+
+def test_sampled_equals_full_backward():
+    rng = np.random.default_rng(7)
+    n, Hq, Hkv = 40, 4, 1
+    q = rng.standard_normal((n, Hq, 6))
+    k = rng.standard_normal((n, Hkv, 6))
+    v = rng.standard_normal((n, Hkv, 2))
+    s = rng.standard_normal(Hq)
+    W = rng.standard_normal((n, Hq, 2))
+    for window in (0, 7):
+        dq, dk, dv, ds = prefill_backward(q, k, v, W, s, window, np.array([0, n]))
+        rows = list(range(n))
+        sq, sk, sv, ss = oracle.backward.prefill_backward_sampled(
+            q, k, v, W, s, window, rows, list(range(Hq)), rows, [0], sink_heads=list(range(Hq)), block=16)
+        np.testing.assert_allclose(sq, dq, atol=1e-12)
+        np.testing.assert_allclose(sk, dk, atol=1e-12)
+        np.testing.assert_allclose(sv, dv, atol=1e-12)
+        np.testing.assert_allclose(ss, ds, atol=1e-12)
