@@ -418,8 +418,9 @@ def run_ours(args, rank, world, peaks, peak_kind):
             "ms": round(m_b, 3), "TFLOP/s": round(fb / (m_b * 1e-3) / 1e12, 1),
             "roofline_frac": round(fb / (m_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
             "bound": "tensor", "useful_flop": fb, "launches": 5,
-            "note": "dq, dk, dv, dsinks with warp-level mma.sync (the forward's out and lse as "
-                    "inputs); the dV pass recomputes S"}
+            "note": "dq, dk, dv, dsinks with warp-level mma.sync, cp.async double-buffered tiles "
+                    "(the forward's out and lse as inputs); the dQ and dK passes recompute S and dP, "
+                    "the dV pass S"}
         del xb, ob, lb, dob
 
     res = {
@@ -620,7 +621,17 @@ def run_case(args):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     T = args.seq_len
-    if args.case.startswith("prefill"):
+    if args.case == "prefill_backward":
+        # one global layer's backward (its forward runs once, untimed)
+        x = W.prefill_inputs([T], seed=1, device=dev)
+        o, l = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, 0, x.cu_seqlens, T)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2)
+        do = torch.randn(o.shape, generator=gen, device=dev).to(o.dtype)
+        fn = lambda: mimo.mimo_attn_prefill_backward(x.q, x.k, x.v, o, l, do, x.sinks, 0,  # noqa: E731
+                                                      x.cu_seqlens, T)
+        work = (1664 * HQ * (T * (T + 1) // 2), 0)
+    elif args.case.startswith("prefill"):
         window = SWA if args.case == "prefill_swa" else 0
         x = W.prefill_inputs([T], seed=1, device=dev)
         out = torch.empty((T, HQ, DV), dtype=torch.bfloat16, device=dev)
@@ -680,7 +691,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the FP8-cache decode measured after the step")
     ap.add_argument("--case", choices=["step", "prefill_swa", "prefill_global", "decode_global",
-                                       "decode_ring", "decode_global_fp8"], default="step",
+                                       "decode_ring", "decode_global_fp8", "prefill_backward"],
+                    default="step",
                     help="run one kernel alone (profiling); 'step' is the benchmark")
     ap.add_argument("--seq-len", type=int, default=T_PREFILL, help="prefill length for --case")
     ap.add_argument("--decode-cap", type=int, default=0,
