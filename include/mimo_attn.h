@@ -216,8 +216,19 @@ size_t mimo_attn_prefill_backward_workspace_size(const mimo_attn_dims_t* dims,
  *   workspace  >= mimo_attn_prefill_backward_workspace_size() bytes, 16-byte aligned
  *
  * Warp-level tensor-core kernels (mma.sync, bf16 operands, fp32
- * accumulation; P and dS rounded to bf16 as operands); deterministic: no
- * atomics.
+ * accumulation; P, dS and dO rounded to bf16 as operands, fp32 dO included,
+ * and D computed from that rounded dO); deterministic: no atomics, fixed
+ * summation order.
+ *
+ * All buffers are caller-owned device memory; the call is asynchronous on
+ * `stream`.  Errors, returned before any launch: the dims rules of
+ * mimo_attn_prefill (MIMO_ERR_UNSUPPORTED / MIMO_ERR_INVALID_ARG); window < 0,
+ * negative sizes, cu_seqlens NULL, any of q, k, v, out, lse, dout, dq, dk, dv
+ * NULL, dsinks NULL while sinks is given, tensors not 16-byte aligned (lse,
+ * sinks, dsinks 4-byte), or max_seqlen > total_tokens -> MIMO_ERR_INVALID_ARG;
+ * num_seqs > 65535 -> MIMO_ERR_UNSUPPORTED; a missing or small workspace ->
+ * MIMO_ERR_WORKSPACE.  total_tokens, num_seqs or max_seqlen of 0 is a no-op
+ * returning MIMO_OK.  max_seqlen must be at least the longest sequence.
  */
 mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const void* q,
                                          const void* k, const void* v, const void* out,
