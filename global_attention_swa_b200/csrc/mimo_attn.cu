@@ -17,6 +17,7 @@
 #include "rope_append_kernel.cuh"
 #include "decode_merge_kernel.cuh"
 #include "backward_kernel.cuh"
+#include "backward_tc_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
@@ -151,6 +152,11 @@ mimo_status_t ensure_attributes() {
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kBkSmemBytes),
                        "backward dv smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_tc_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::kBtSmemBytes),
+                       "backward dk/dv (tcgen05) smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dkv_kernel<false>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -641,6 +647,41 @@ mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const voi
   const int qtiles = (max_seqlen + mimo::kBqRows - 1) / mimo::kBqRows;
   mimo::bwd_dq_kernel<<<dim3(qtiles, p.Hq, num_seqs), mimo::kBkThreads, mimo::kBqSmemBytes, s>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "backward dq launch"))) return st;
+  if (!p.io_f32) {
+    // bf16 out / dout: dK and dV in one tcgen05 pass over 128-key tiles
+    CUtensorMap tq, tk, tv, tdo;
+    const int Hq = p.Hq, Hkv = p.Hkv;
+    {
+      const uint64_t d[3] = {192, (uint64_t)Hq, (uint64_t)total_tokens};
+      const uint64_t st2[2] = {192 * 2, (uint64_t)Hq * 192 * 2};
+      const uint32_t b[3] = {64, 1, mimo::kBtQ};
+      if ((st = make_map(&tq, q, 3, d, st2, b))) return st;
+    }
+    {
+      const uint64_t d[3] = {128, (uint64_t)Hq, (uint64_t)total_tokens};
+      const uint64_t st2[2] = {128 * 2, (uint64_t)Hq * 128 * 2};
+      const uint32_t b[3] = {64, 1, mimo::kBtQ};
+      if ((st = make_map(&tdo, dout, 3, d, st2, b))) return st;
+    }
+    {
+      const uint64_t d[3] = {192, (uint64_t)Hkv, (uint64_t)total_tokens};
+      const uint64_t st2[2] = {192 * 2, (uint64_t)Hkv * 192 * 2};
+      const uint32_t b[3] = {64, 1, mimo::kBtKeys};
+      if ((st = make_map(&tk, k, 3, d, st2, b))) return st;
+    }
+    {
+      const uint64_t d[3] = {128, (uint64_t)Hkv, (uint64_t)total_tokens};
+      const uint64_t st2[2] = {128 * 2, (uint64_t)Hkv * 128 * 2};
+      const uint32_t b[3] = {64, 1, mimo::kBtKeys};
+      if ((st = make_map(&tv, v, 3, d, st2, b))) return st;
+    }
+    const int ktiles = (max_seqlen + mimo::kBtKeys - 1) / mimo::kBtKeys;
+    mimo::bwd_dkv_tc_kernel<<<dim3((unsigned)ktiles * Hkv, num_seqs), mimo::kBtThreads, mimo::kBtSmemBytes,
+                              s>>>(tq, tk, tv, tdo, p);
+    if ((st = cuda_check(cudaGetLastError(), "backward dk/dv launch"))) return st;
+    return ok();
+  }
+  // fp32 out / dout: two warp-level passes (dV, then dK)
   const dim3 kv_grid((unsigned)tiles * p.Hkv, num_seqs);  // (key tile, KV head) per CTA
   mimo::bwd_dkv_kernel<true><<<kv_grid, mimo::kBkThreads, mimo::kBkSmemBytes, s>>>(p);
   if ((st = cuda_check(cudaGetLastError(), "backward dv launch"))) return st;

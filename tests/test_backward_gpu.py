@@ -53,16 +53,25 @@ def _run(lengths, hq, hkv, window, sinks, out_dtype, seed, v_scale=1.0):
     return (dq, dk, dv, ds), (rq, rk, rv, rs)
 
 
+# fp32 out / dout take the two warp-level dV and dK passes, bf16 the tcgen05 pass
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("window", [129, 0, 1])
 @pytest.mark.parametrize("sinks", [True, False])
-def test_tiny_heads(window, sinks):
-    got, ref = _run([512], 16, 1, window, sinks, torch.float32, seed=window + 3)
+def test_tiny_heads(window, sinks, io):
+    got, ref = _run([512], 16, 1, window, sinks, io, seed=window + 3)
     for name, a, b in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
         grad_check(a, b, f"{name} W={window}")
     if sinks:
         grad_check(got[3], ref[3], "dsinks")
     else:
         assert got[3] is None
+
+
+def test_small_groups_bf16():
+    """Two query heads per KV head and ragged lengths around the 128-key tile."""
+    got, ref = _run([127, 128, 129, 300], 4, 2, 0, True, torch.bfloat16, seed=21)
+    for name, a, b in zip(("dq", "dk", "dv", "dsinks"), got, ref):
+        grad_check(a, b, name)
 
 
 @pytest.mark.parametrize("window", [129, 0])
@@ -72,9 +81,10 @@ def test_model_heads_varlen_bf16(window):
         grad_check(a, b, f"{name} W={window}")
 
 
-def test_deterministic():
-    a, _ = _run([200, 70], 16, 2, 129, True, torch.float32, seed=5)
-    b, _ = _run([200, 70], 16, 2, 129, True, torch.float32, seed=5)
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_deterministic(io):
+    a, _ = _run([200, 70], 16, 2, 129, True, io, seed=5)
+    b, _ = _run([200, 70], 16, 2, 129, True, io, seed=5)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
 
