@@ -18,7 +18,7 @@
 // and at the end writes dV * v_scale and dK * scale (fp32).
 //
 //   warps 0-3   softmax and epilogue, one key row (TMEM lane) per thread
-//   warp 4      TMA producer (K, V once; Q and dO per item, two stages);
+//   warp 4      TMA producer (K, V once; Q and dO per item, three stages);
 //               allocates / frees the 512 TMEM columns
 //   warp 5      MMA issuer (one thread)
 //
@@ -44,8 +44,9 @@ constexpr int kBtOBytes = 64 * 128 * 2;       // 2 boxes (dO)
 constexpr int kBtStage = kBtQBytes + kBtOBytes;
 constexpr int kBtOffK = 0;
 constexpr int kBtOffV = kBtKBytes;
-constexpr int kBtOffStage = kBtOffV + kBtVBytes;          // 2 stages
-constexpr int kBtOffLD = kBtOffStage + 2 * kBtStage;      // 2 x {lse log2e [64], D [64]}
+constexpr int kBtStages = 3;
+constexpr int kBtOffStage = kBtOffV + kBtVBytes;
+constexpr int kBtOffLD = kBtOffStage + kBtStages * kBtStage;  // 2 x {lse log2e [64], D [64]}
 constexpr int kBtOffBar = kBtOffLD + 2 * 2 * kBtQ * 4;
 constexpr int kBtSmemBytes = kBtOffBar + 128 + 1024;      // barriers + alignment slack
 constexpr uint32_t kBtColDV = 0, kBtColDK = 128, kBtColS0 = 320, kBtColDP = 384, kBtColS1 = 448;
@@ -58,14 +59,14 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBtOffBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;   // [2]
-  uint64_t* q_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* p_full = bars + 6;
-  uint64_t* ld_full = bars + 7;  // [2]
-  uint64_t* done = bars + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 11);
+  uint64_t* q_full = bars + 1;   // [kBtStages]
+  uint64_t* q_empty = bars + 4;  // [kBtStages]
+  uint64_t* s_full = bars + 7;
+  uint64_t* p_full = bars + 8;
+  uint64_t* ld_full = bars + 9;  // [2]
+  uint64_t* done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
   float* sLD = reinterpret_cast<float*>(smem + kBtOffLD);
 
   // key tiles in ascending order, KV heads fastest: the longest causal loops start first
@@ -83,11 +84,11 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   if (warp == 4) {
     if (lane == 0) {
       mbar_init(kv_full, 1);
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < kBtStages; ++i) {
         mbar_init(&q_full[i], 1);
         mbar_init(&q_empty[i], 1);
-        mbar_init(&ld_full[i], 128);
       }
+      for (int i = 0; i < 2; ++i) mbar_init(&ld_full[i], 128);
       mbar_init(s_full, 1);
       mbar_init(p_full, 128);
       mbar_init(done, 1);
@@ -119,8 +120,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) tma_load_3d(smem + kBtOffV + c * 16384, &tm_v, kv_full, c * 64, g, b0 + k0);
       for (int j = 0; j < items; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !wait_bounded(&q_empty[st], ((j >> 1) - 1) & 1, abort_flag)) break;
+        const int st = j % kBtStages;
+        if (j >= kBtStages && !wait_bounded(&q_empty[st], (j / kBtStages - 1) & 1, abort_flag)) break;
         const int h = g * p.G + j / nq;
         const int row = b0 + (qt_lo + j % nq) * kBtQ;
         uint8_t* stg = smem + kBtOffStage + st * kBtStage;
@@ -185,19 +186,20 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         umma_commit(s_full);
       }
       for (int j = 0; ok && j < items; ++j) {
-        const int st = j & 1;
+        const int st = j % kBtStages;
+        const int sn = (j + 1) % kBtStages;
         const bool more = j + 1 < items;
         if (more) {
-          if (!(ok = wait_bounded(&q_full[st ^ 1], ((j + 1) >> 1) & 1, abort_flag))) break;
+          if (!(ok = wait_bounded(&q_full[sn], ((j + 1) / kBtStages) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_s(tS(j + 1), st ^ 1);  // overlaps the softmax of item j
+          issue_s(tS(j + 1), sn);  // overlaps the softmax of item j
         }
         if (!(ok = wait_bounded(p_full, j & 1, abort_flag))) break;
         tc_fence_after();
         issue_acc(j, st);
         umma_commit(&q_empty[st]);
         if (more) {
-          issue_dp(st ^ 1);
+          issue_dp(sn);
           umma_commit(s_full);
         }
       }
@@ -208,22 +210,22 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     const int r = threadIdx.x;  // TMEM lane == key row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int key = k0 + r;
+    // one value per thread of each item's lse (base 2, threads 0-63) or D
+    // (threads 64-127), loaded one item ahead and passed on through shared memory
+    auto fetch = [&](int j) -> float {
+      const int qp = (qt_lo + j % nq) * kBtQ + (r & (kBtQ - 1));
+      if (qp >= len) return 0.f;
+      const size_t gi = (size_t)(g * p.G + j / nq) * p.total + b0 + qp;
+      return r < kBtQ ? p.lse[gi] * 1.4426950408889634f : p.D[gi];
+    };
     bool ok = items > 0;
+    float nxt = ok ? fetch(0) : 0.f;
     for (int j = 0; ok && j < items; ++j) {
-      const int h = g * p.G + j / nq;
       const int q0 = (qt_lo + j % nq) * kBtQ;
-      // this item's lse (base 2) and D, one value per thread, through shared memory
       float* ld = sLD + (j & 1) * 2 * kBtQ;
-      {
-        const int c = r & (kBtQ - 1);
-        const int qp = q0 + c;
-        const size_t gi = (size_t)h * p.total + b0 + qp;
-        if (r < kBtQ)
-          ld[c] = qp < len ? p.lse[gi] * 1.4426950408889634f : 0.f;
-        else
-          ld[kBtQ + c] = qp < len ? p.D[gi] : 0.f;
-      }
+      ld[r] = nxt;
       mbar_arrive(&ld_full[j & 1]);
+      if (j + 1 < items) nxt = fetch(j + 1);  // in flight during this item
       if (!(ok = wait_bounded(&ld_full[j & 1], (j >> 1) & 1, abort_flag))) break;
       if (!(ok = wait_bounded(s_full, j & 1, abort_flag))) break;
       tc_fence_after();
