@@ -417,10 +417,10 @@ def run_ours(args, rank, world, peaks, peak_kind):
         extra["prefill_backward_global_T8192"] = {
             "ms": round(m_b, 3), "TFLOP/s": round(fb / (m_b * 1e-3) / 1e12, 1),
             "roofline_frac": round(fb / (m_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
-            "bound": "tensor", "useful_flop": fb, "launches": 5,
-            "note": "dq, dk, dv, dsinks with warp-level mma.sync, cp.async double-buffered tiles "
-                    "(the forward's out and lse as inputs); the dQ and dK passes recompute S and dP, "
-                    "the dV pass S"}
+            "bound": "tensor", "useful_flop": fb, "launches": 4,
+            "note": "dq, dk, dv, dsinks (the forward's out and lse as inputs): dK and dV in one "
+                    "tcgen05 pass, dQ with warp-level mma.sync (recomputing S and dP), D and the "
+                    "sink gradient in two small launches"}
         del xb, ob, lb, dob
 
     res = {
