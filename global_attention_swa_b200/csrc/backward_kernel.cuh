@@ -8,8 +8,8 @@
 //   dq_i = s sum_j dS_ij k_j;  dk_j = s sum_{h in group, i} dS_ij q_i;
 //   dv_j = v_scale sum_{h in group, i} P_ij dO_i;  dsigma_h = -sum_i exp(sigma_h - lse_i) D_i
 //
-// Five launches, warp-level mma.sync m16n8k16 (bf16 in, fp32 accumulate; P
-// and dS rounded to bf16 as operands):
+// The kernels here (warp-level mma.sync m16n8k16: bf16 in, fp32 accumulate;
+// P and dS rounded to bf16 as operands):
 //   bwd_preprocess_kernel  D and the sink terms, one warp per (token, head)
 //   bwd_sink_kernel        dsigma_h, one CTA per head (deterministic sum)
 //   bwd_dq_kernel          CTA per (128-query tile, head): loops over key tiles
@@ -17,10 +17,12 @@
 //   bwd_dkv_kernel<DV>     CTA per (64-key tile, KV head): loops over the
 //   bwd_dkv_kernel<DK>     group's heads and query tiles (double-buffered);
 //                          dV and dK in two passes (each accumulator alone
-//                          fits the registers)
+//                          fits the registers).  Used for fp32 out / dout;
+//                          with bf16 ones dK and dV come from the tcgen05
+//                          kernel in backward_tc_kernel.cuh.
 // Tiles of 64 rows sit in shared memory with a 16-byte-chunk XOR swizzle
 // (chunk ^ row % 8) so that ldmatrix reads are conflict-free.  No kernel
-// waits on another thread beyond __syncthreads.
+// here waits on another thread beyond __syncthreads.
 #pragma once
 
 #include "common.cuh"

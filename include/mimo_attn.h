@@ -215,9 +215,10 @@ size_t mimo_attn_prefill_backward_workspace_size(const mimo_attn_dims_t* dims,
  *   dsinks     [Hq] fp32, required when sinks is given (ignored otherwise)
  *   workspace  >= mimo_attn_prefill_backward_workspace_size() bytes, 16-byte aligned
  *
- * Warp-level tensor-core kernels (mma.sync, bf16 operands, fp32
- * accumulation; P, dS and dO rounded to bf16 as operands, fp32 dO included,
- * and D computed from that rounded dO); deterministic: no atomics, fixed
+ * Tensor-core kernels with bf16 operands and fp32 accumulation (dK and dV
+ * on tcgen05 when out / dout are bf16, warp-level mma.sync otherwise and for
+ * dq); P, dS and dO are rounded to bf16 as operands (fp32 dO included) and D
+ * is computed from that rounded dO; deterministic: no atomics, fixed
  * summation order.
  *
  * All buffers are caller-owned device memory; the call is asynchronous on
