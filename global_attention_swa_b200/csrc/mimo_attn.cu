@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -172,17 +173,19 @@ mimo_status_t ensure_attributes() {
   return MIMO_OK;
 }
 
+// SMs of the current device (148 on B200; also the answer without a device,
+// so that host-only size queries match the launches on B200).
 int sm_count() {
-  static int counts[64] = {0};
+  static std::atomic<int> counts[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!counts[dev]) {
-    int c = 0;
+  int c = counts[dev].load(std::memory_order_relaxed);
+  if (c <= 0) {
     if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
       c = 148;
-    counts[dev] = c;
+    counts[dev].store(c, std::memory_order_relaxed);
   }
-  return counts[dev];
+  return c;
 }
 
 // ---------------------------------------------------------------- decode plan
@@ -214,7 +217,7 @@ DecodePlan decode_plan(int batch, int hkv, int capacity, int window) {
   int chunk = env_chunk();
   if (chunk <= 0) {
     const long units = (long)batch * hkv;
-    const long want = 2L * 148;
+    const long want = 2L * sm_count();
     long nsplit = (want + units - 1) / units;
     long max_split = std::max(1L, ((long)pl.cap_eff + 255) / 256);
     nsplit = std::max(1L, std::min(nsplit, max_split));

@@ -98,6 +98,13 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims,
 /*
  * Bytes of device workspace mimo_attn_decode needs for these sizes
  * (split-KV partial results).  0 when one split covers every sequence.
+ *
+ * The split plan depends only on these sizes and the current device's SM
+ * count (148 on B200, also assumed when no device is visible): about two
+ * work units per SM, splits of 256..16384 keys, one split for a ring cache.
+ * For tuning, the environment variable MIMO_DECODE_CHUNK (keys per split,
+ * rounded up to a multiple of 64; read once per process) overrides the split
+ * size; this size query and the decode call then follow the same plan.
  */
 size_t mimo_attn_decode_workspace_size(const mimo_attn_dims_t* dims, int batch,
                                        int capacity, int window);
