@@ -115,8 +115,23 @@ def _check(status):
         raise MimoAttnError(status, lib.mimo_attn_last_error().decode())
 
 
-def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+_BF16, _F32, _I32 = torch.bfloat16, torch.float32, torch.int32
+_OUT = (torch.bfloat16, torch.float32)
+
+
+def _ptr(t, name="tensor", dtype=None):
+    """Device address of a contiguous CUDA tensor (None for None).  The C ABI takes
+    plain pointers, so a host tensor, a strided view or another dtype would be
+    read as garbage: each is refused here."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
@@ -146,9 +161,11 @@ def mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, out=None, 
     if lse is None and return_lse:
         lse = torch.empty((hq, nt), dtype=torch.float32, device=q.device)
     dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
-    _check(lib.mimo_attn_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(sinks),
-                                 int(window), _ptr(cu_seqlens), int(cu_seqlens.numel() - 1), nt,
-                                 int(max_seqlen), _ptr(out), _ptr(lse), _stream(stream)))
+    _check(lib.mimo_attn_prefill(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16),
+                                 _ptr(v, "v", _BF16), _ptr(sinks, "sinks", _F32), int(window),
+                                 _ptr(cu_seqlens, "cu_seqlens", _I32), int(cu_seqlens.numel() - 1), nt,
+                                 int(max_seqlen), _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
+                                 _stream(stream)))
     return out, lse
 
 
@@ -176,9 +193,11 @@ def mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, out=None, lse=
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                _ptr(seqlens), B, C, int(window), _ptr(sinks), _ptr(out),
-                                _ptr(lse), _ptr(workspace), wbytes, _stream(stream)))
+    _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_cache, "k_cache", _BF16),
+                                _ptr(v_cache, "v_cache", _BF16), _ptr(seqlens, "seqlens", _I32), B, C,
+                                int(window), _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                _ptr(lse, "lse", _F32), _ptr(workspace, "workspace"), wbytes,
+                                _stream(stream)))
     return out, lse
 
 
@@ -204,10 +223,12 @@ def mimo_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale_kv, seqlens, wind
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.mimo_attn_decode_fp8(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                    _ptr(k_scale), _ptr(v_scale_kv), _ptr(seqlens), B, C,
-                                    int(window), _ptr(sinks), _ptr(out), _ptr(lse),
-                                    _ptr(workspace), wbytes, _stream(stream)))
+    _check(lib.mimo_attn_decode_fp8(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_cache, "k_cache"),
+                                    _ptr(v_cache, "v_cache"), _ptr(k_scale, "k_scale", _F32),
+                                    _ptr(v_scale_kv, "v_scale_kv", _F32), _ptr(seqlens, "seqlens", _I32),
+                                    B, C, int(window), _ptr(sinks, "sinks", _F32),
+                                    _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
+                                    _ptr(workspace, "workspace"), wbytes, _stream(stream)))
     return out, lse
 
 
@@ -219,9 +240,10 @@ def mimo_attn_rope_append(q, k_new, v_new, k_cache, v_cache, seqlens, window, ro
     C, hkv = k_cache.shape[1], k_cache.shape[2]
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3])
     rd = dqk if rotary_dim is None else int(rotary_dim)
-    _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new),
-                                     _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, C,
-                                     int(window), float(rope_theta), rd, _stream(stream)))
+    _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_new, "k_new", _BF16),
+                                     _ptr(v_new, "v_new", _BF16), _ptr(k_cache, "k_cache", _BF16),
+                                     _ptr(v_cache, "v_cache", _BF16), _ptr(seqlens, "seqlens", _I32),
+                                     B, C, int(window), float(rope_theta), rd, _stream(stream)))
     return q
 
 
@@ -235,8 +257,9 @@ def mimo_attn_decode_merge(part_out, part_lse, sinks, out=None, lse=None,
     if lse is None and return_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=part_out.device)
     dims = make_dims(hq, 1, 192, dv, None, v_scale, out.dtype)
-    _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out), _ptr(part_lse), R, B,
-                                      _ptr(sinks), _ptr(out), _ptr(lse), _stream(stream)))
+    _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out, "part_out", _F32),
+                                      _ptr(part_lse, "part_lse", _F32), R, B, _ptr(sinks, "sinks", _F32),
+                                      _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32), _stream(stream)))
     return out, lse
 
 
@@ -255,9 +278,11 @@ def mimo_attn_prefill_backward(q, k, v, out, lse, dout, sinks, window, cu_seqlen
     dims = make_dims(hq, hkv, dqk, dv_dim, softmax_scale, v_scale, out.dtype)
     need = int(lib.mimo_attn_prefill_backward_workspace_size(ctypes.byref(dims), nt))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _check(lib.mimo_attn_prefill_backward(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                                          _ptr(lse), _ptr(dout), _ptr(sinks), int(window),
-                                          _ptr(cu_seqlens), cu_seqlens.numel() - 1, nt,
+    _check(lib.mimo_attn_prefill_backward(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16),
+                                          _ptr(v, "v", _BF16), _ptr(out, "out", _OUT),
+                                          _ptr(lse, "lse", _F32), _ptr(dout, "dout", out.dtype),
+                                          _ptr(sinks, "sinks", _F32), int(window),
+                                          _ptr(cu_seqlens, "cu_seqlens", _I32), cu_seqlens.numel() - 1, nt,
                                           int(max_seqlen), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds),
                                           _ptr(ws), ws.numel(), _stream(stream)))
     return dq, dk, dv, ds
@@ -281,7 +306,9 @@ def mimo_attn_decode_noalloc(q, k_cache, v_cache, seqlens, window, sinks, out, l
     B, hq, dqk = q.shape
     C, hkv = k_cache.shape[1], k_cache.shape[2]
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3], softmax_scale, v_scale, out.dtype)
-    _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                        _ptr(seqlens), B, C, int(window), _ptr(sinks), _ptr(out),
-                                        _ptr(lse), _stream(stream)))
+    _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                        _ptr(k_cache, "k_cache", _BF16), _ptr(v_cache, "v_cache", _BF16),
+                                        _ptr(seqlens, "seqlens", _I32), B, C, int(window),
+                                        _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                        _ptr(lse, "lse", _F32), _stream(stream)))
     return out, lse

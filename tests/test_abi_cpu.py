@@ -174,3 +174,98 @@ def test_prefill_backward_rejects_bad_arguments():
 def test_last_error_is_empty_after_success():
     assert _prefill(_dims(), total=0, maxlen=0) == mimo.MIMO_OK
     assert mimo.lib.mimo_attn_last_error().decode() == ""
+
+
+def test_binding_refuses_tensors_it_cannot_pass_as_plain_pointers():
+    """The binding passes raw device addresses: host tensors, strided views and
+    wrong dtypes are refused before the library is called."""
+    import types
+
+    import torch
+
+    assert mimo._ptr(None) is None
+    with pytest.raises(ValueError, match="CUDA"):
+        mimo._ptr(torch.zeros(4), "x")
+    fake = lambda contig, dt: types.SimpleNamespace(  # noqa: E731
+        is_cuda=True, is_contiguous=lambda: contig, dtype=dt, data_ptr=lambda: 4096)
+    with pytest.raises(ValueError, match="contiguous"):
+        mimo._ptr(fake(False, torch.bfloat16), "q", torch.bfloat16)
+    with pytest.raises(TypeError, match="q must be"):
+        mimo._ptr(fake(True, torch.float16), "q", torch.bfloat16)
+    with pytest.raises(TypeError):
+        mimo._ptr(fake(True, torch.float16), "out", (torch.bfloat16, torch.float32))
+    assert mimo._ptr(fake(True, torch.float32), "out", (torch.bfloat16, torch.float32)).value == 4096
+    # a wrapper given host tensors fails in the binding, not in the library
+    q = torch.zeros((8, 4, 192), dtype=torch.bfloat16)
+    k = torch.zeros((8, 1, 192), dtype=torch.bfloat16)
+    v = torch.zeros((8, 1, 128), dtype=torch.bfloat16)
+    cu = torch.tensor([0, 8], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        mimo.mimo_attn_prefill(q, k, v, None, 0, cu, 8)
+
+
+def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
+    """Dry run of each wrapper on host tensors of the documented dtypes against a
+    stand-in library that records its calls (the device check alone is bypassed):
+    argument checks and marshalling raise nothing for valid inputs."""
+    import types
+
+    import torch
+
+    calls = []
+
+    class FakeLib:
+        def __getattr__(self, name):
+            def fn(*args):
+                calls.append(name)
+                return 0
+            return fn
+
+    real_ptr = mimo._ptr
+
+    def host_ptr(t, name="tensor", dtype=None):
+        if t is None:
+            return None
+        proxy = types.SimpleNamespace(is_cuda=True, is_contiguous=t.is_contiguous, dtype=t.dtype,
+                                      data_ptr=t.data_ptr)
+        return real_ptr(proxy, name, dtype)
+
+    monkeypatch.setattr(mimo, "lib", FakeLib())
+    monkeypatch.setattr(mimo, "_ptr", host_ptr)
+    monkeypatch.setattr(mimo, "_stream", lambda stream: None)
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    B, C, Hq, Hkv, Nt = 2, 16, 4, 1, 24
+    q = torch.zeros((Nt, Hq, 192), dtype=bf)
+    k = torch.zeros((Nt, Hkv, 192), dtype=bf)
+    v = torch.zeros((Nt, Hkv, 128), dtype=bf)
+    sinks = torch.zeros(Hq, dtype=f32)
+    cu = torch.tensor([0, 10, 24], dtype=i32)
+    for odt in (bf, f32):
+        out, lse = mimo.mimo_attn_prefill(q, k, v, sinks, 129, cu, 14, out_dtype=odt)
+        assert out.dtype == odt and lse.dtype == f32
+        dout = torch.zeros_like(out)
+        dq, dk, dv, ds = mimo.mimo_attn_prefill_backward(q, k, v, out, lse, dout, sinks, 0, cu, 14)
+        assert dq.shape == q.shape and dk.shape == k.shape and dv.shape == v.shape
+        with pytest.raises(TypeError):
+            mimo.mimo_attn_prefill_backward(q, k, v, out, lse, dout.to(f32 if odt == bf else bf),
+                                            sinks, 0, cu, 14)
+    qd = torch.zeros((B, Hq, 192), dtype=bf)
+    kc = torch.zeros((B, C, Hkv, 192), dtype=bf)
+    vc = torch.zeros((B, C, Hkv, 128), dtype=bf)
+    sl = torch.tensor([3, 16], dtype=i32)
+    mimo.mimo_attn_decode(qd, kc, vc, sl, 0, sinks)
+    mimo.mimo_attn_decode(qd, kc, vc, sl, 0, None, out_dtype=f32)
+    codes_k = torch.zeros((B, C, Hkv, 192), dtype=torch.uint8)
+    codes_v = torch.zeros((B, C, Hkv, 128), dtype=torch.uint8)
+    scale = torch.ones(Hkv, dtype=f32)
+    mimo.mimo_attn_decode_fp8(qd, codes_k, codes_v, scale, scale, sl, 0, sinks)
+    mimo.mimo_attn_rope_append(qd, torch.zeros((B, Hkv, 192), dtype=bf), torch.zeros((B, Hkv, 128), dtype=bf),
+                               kc, vc, sl, 16, 10000.0)
+    mimo.mimo_attn_decode_merge(torch.zeros((3, B, Hq, 128)), torch.zeros((3, B, Hq)), sinks)
+    mimo.mimo_attn_decode_noalloc(qd, kc, vc, sl, 0, sinks, torch.zeros((B, Hq, 128), dtype=bf))
+    with pytest.raises(TypeError, match="seqlens"):
+        mimo.mimo_attn_decode(qd, kc, vc, sl.long(), 0, sinks)
+    with pytest.raises(ValueError, match="contiguous"):
+        mimo.mimo_attn_decode(qd, kc[:, ::2], vc[:, ::2], sl, 0, sinks)
+    assert {"mimo_attn_prefill", "mimo_attn_prefill_backward", "mimo_attn_decode", "mimo_attn_decode_fp8",
+            "mimo_attn_rope_append", "mimo_attn_decode_merge", "mimo_attn_decode_noalloc"} <= set(calls)
