@@ -134,6 +134,13 @@ def _ptr(t, name="tensor", dtype=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _shape(t, shape, name):
+    """Refuse a tensor whose shape disagrees with the sizes the call derives from
+    its other arguments (the library would read or write past its end)."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -156,6 +163,13 @@ def mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, out=None, 
     """
     nt, hq, dqk = q.shape
     hkv, dv = k.shape[1], v.shape[2]
+    _shape(k, (nt, hkv, dqk), "k")
+    _shape(v, (nt, hkv, dv), "v")
+    _shape(sinks, (hq,), "sinks")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be 1-D with num_seqs + 1 entries")
+    _shape(out, (nt, hq, dv), "out")
+    _shape(lse, (hq, nt), "lse")
     if out is None:
         out = torch.empty((nt, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
@@ -167,6 +181,19 @@ def mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, out=None, 
                                  int(max_seqlen), _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
                                  _stream(stream)))
     return out, lse
+
+
+def _decode_shapes(q, k_cache, v_cache, seqlens, sinks, out, lse):
+    B, hq, dqk = q.shape
+    if k_cache.dim() != 4 or v_cache.dim() != 4:
+        raise ValueError("caches must be [batch, capacity, Hkv, D]")
+    C, hkv = k_cache.shape[1], k_cache.shape[2]
+    _shape(k_cache, (B, C, hkv, dqk), "k_cache")
+    _shape(v_cache, (B, C, hkv, v_cache.shape[3]), "v_cache")
+    _shape(seqlens, (B,), "seqlens")
+    _shape(sinks, (hq,), "sinks")
+    _shape(out, (B, hq, v_cache.shape[3]), "out")
+    _shape(lse, (B, hq), "lse")
 
 
 def mimo_attn_decode_workspace_size(hq, hkv, batch, capacity, window, dqk=192, dv=128):
@@ -184,6 +211,7 @@ def mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, out=None, lse=
     B, hq, dqk = q.shape
     C, hkv = k_cache.shape[1], k_cache.shape[2]
     dv = v_cache.shape[3]
+    _decode_shapes(q, k_cache, v_cache, seqlens, sinks, out, lse)
     if out is None:
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
@@ -214,6 +242,9 @@ def mimo_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale_kv, seqlens, wind
     dv = v_cache.shape[3]
     if k_cache.element_size() != 1 or v_cache.element_size() != 1:
         raise TypeError("FP8 caches hold one byte per element")
+    _decode_shapes(q, k_cache, v_cache, seqlens, sinks, out, lse)
+    _shape(k_scale, (hkv,), "k_scale")
+    _shape(v_scale_kv, (hkv,), "v_scale_kv")
     if out is None:
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
@@ -238,6 +269,9 @@ def mimo_attn_rope_append(q, k_new, v_new, k_cache, v_cache, seqlens, window, ro
     position seqlens - 1 (see include/mimo_attn.h).  Returns q."""
     B, hq, dqk = q.shape
     C, hkv = k_cache.shape[1], k_cache.shape[2]
+    _decode_shapes(q, k_cache, v_cache, seqlens, None, None, None)
+    _shape(k_new, (B, hkv, dqk), "k_new")
+    _shape(v_new, (B, hkv, v_cache.shape[3]), "v_new")
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3])
     rd = dqk if rotary_dim is None else int(rotary_dim)
     _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_new, "k_new", _BF16),
@@ -252,6 +286,10 @@ def mimo_attn_decode_merge(part_out, part_lse, sinks, out=None, lse=None,
     """Merge per-part decode results (part_out [R,B,Hq,128] fp32, part_lse [R,B,Hq] fp32)
     with the sink.  Returns (out [B,Hq,128], lse [B,Hq] or None)."""
     R, B, hq, dv = part_out.shape
+    _shape(part_lse, (R, B, hq), "part_lse")
+    _shape(sinks, (hq,), "sinks")
+    _shape(out, (B, hq, dv), "out")
+    _shape(lse, (B, hq), "lse")
     if out is None:
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=part_out.device)
     if lse is None and return_lse:
@@ -271,6 +309,14 @@ def mimo_attn_prefill_backward(q, k, v, out, lse, dout, sinks, window, cu_seqlen
     """
     nt, hq, dqk = q.shape
     hkv, dv_dim = k.shape[1], v.shape[2]
+    _shape(k, (nt, hkv, dqk), "k")
+    _shape(v, (nt, hkv, dv_dim), "v")
+    _shape(out, (nt, hq, dv_dim), "out")
+    _shape(lse, (hq, nt), "lse")
+    _shape(dout, (nt, hq, dv_dim), "dout")
+    _shape(sinks, (hq,), "sinks")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be 1-D with num_seqs + 1 entries")
     dq = torch.empty((nt, hq, dqk), dtype=torch.float32, device=q.device)
     dk = torch.empty((nt, hkv, dqk), dtype=torch.float32, device=q.device)
     dv = torch.empty((nt, hkv, dv_dim), dtype=torch.float32, device=q.device)
@@ -305,6 +351,7 @@ def mimo_attn_decode_noalloc(q, k_cache, v_cache, seqlens, window, sinks, out, l
     """
     B, hq, dqk = q.shape
     C, hkv = k_cache.shape[1], k_cache.shape[2]
+    _decode_shapes(q, k_cache, v_cache, seqlens, sinks, out, lse)
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3], softmax_scale, v_scale, out.dtype)
     _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q, "q", _BF16),
                                         _ptr(k_cache, "k_cache", _BF16), _ptr(v_cache, "v_cache", _BF16),

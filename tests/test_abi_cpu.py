@@ -265,6 +265,17 @@ def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
     mimo.mimo_attn_decode_noalloc(qd, kc, vc, sl, 0, sinks, torch.zeros((B, Hq, 128), dtype=bf))
     with pytest.raises(TypeError, match="seqlens"):
         mimo.mimo_attn_decode(qd, kc, vc, sl.long(), 0, sinks)
+    # sizes that disagree with the ones derived from q would be read past their end
+    with pytest.raises(ValueError, match="k has shape"):
+        mimo.mimo_attn_prefill(q, k[:-1], v, sinks, 0, cu, 14)
+    with pytest.raises(ValueError, match="v_cache"):
+        mimo.mimo_attn_decode(qd, kc, vc[:1], sl, 0, sinks)
+    with pytest.raises(ValueError, match="seqlens"):
+        mimo.mimo_attn_decode(qd, kc, vc, sl[:1], 0, sinks)
+    with pytest.raises(ValueError, match="sinks"):
+        mimo.mimo_attn_decode(qd, kc, vc, sl, 0, torch.zeros(Hq + 1))
+    with pytest.raises(ValueError, match="part_lse"):
+        mimo.mimo_attn_decode_merge(torch.zeros((3, B, Hq, 128)), torch.zeros((2, B, Hq)), sinks)
     with pytest.raises(ValueError, match="contiguous"):
         mimo.mimo_attn_decode(qd, kc[:, ::2], vc[:, ::2], sl, 0, sinks)
     assert {"mimo_attn_prefill", "mimo_attn_prefill_backward", "mimo_attn_decode", "mimo_attn_decode_fp8",
