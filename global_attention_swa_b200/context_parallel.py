@@ -49,9 +49,12 @@ def context_parallel_decode(q, k_cache, v_cache, part_lens, sinks, group=None,
     local_part = local_part or _local_part_cuda
     merge = merge or _merge_cuda
     part_out, part_lse = local_part(q, k_cache, v_cache, part_lens, softmax_scale)
+    B, hq, dv = part_out.shape
+    # one exchange: each rank's (out, lse) packed as [B, Hq, Dv + 1]
+    packed = torch.cat([part_out.reshape(B, hq, dv), part_lse.reshape(B, hq, 1).to(part_out.dtype)],
+                       dim=2).contiguous()
     world = dist.get_world_size(group)
-    outs = [torch.empty_like(part_out) for _ in range(world)]
-    lses = [torch.empty_like(part_lse) for _ in range(world)]
-    dist.all_gather(outs, part_out.contiguous(), group=group)
-    dist.all_gather(lses, part_lse.contiguous(), group=group)
-    return merge(torch.stack(outs), torch.stack(lses), sinks, out_dtype, v_scale)
+    gathered = [torch.empty_like(packed) for _ in range(world)]
+    dist.all_gather(gathered, packed, group=group)
+    g = torch.stack(gathered)
+    return merge(g[..., :dv].contiguous(), g[..., dv].contiguous(), sinks, out_dtype, v_scale)
