@@ -119,3 +119,40 @@ def test_sampled_equals_full_backward():
         np.testing.assert_allclose(sk, dk, atol=1e-12)
         np.testing.assert_allclose(sv, dv, atol=1e-12)
         np.testing.assert_allclose(ss, ds, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [0, 3])
+def test_zero_queries_closed_forms(window):
+    """q = 0: every visible score is 0, so P_ij = 1 / (n_i + e^sigma) with n_i the keys row
+    i sees.  Then O_i = v_scale * mean-like sum, and in closed form
+      dv_j     = v_scale * sum_{i sees j} dO_i / (n_i + e^sigma)
+      dk       = 0                      (dS_ij multiplies q_i = 0)
+      dq_i     = s / (n_i + e^sigma) * sum_{j seen} (v_scale <dO_i, v_j> - D_i) k_j
+      dsigma_h = -sum_i e^sigma / (n_i + e^sigma) * <dO_i, O_i>."""
+    rng = np.random.default_rng(60 + window)
+    n, Hq, Hkv, Dqk, Dv = 7, 2, 1, 4, 3
+    q = np.zeros((n, Hq, Dqk))
+    k = rng.standard_normal((n, Hkv, Dqk))
+    v = rng.standard_normal((n, Hkv, Dv))
+    s = np.array([0.4, -1.1])
+    dO = rng.standard_normal((n, Hq, Dv))
+    vs = 0.8
+    dq, dk, dv, ds = prefill_backward(q, k, v, dO, s, window, np.array([0, n]), scale=0.5, v_scale=vs)
+    np.testing.assert_array_equal(dk, 0.0)
+    want_dv = np.zeros((n, Hkv, Dv))
+    want_dq = np.zeros((n, Hq, Dqk))
+    want_ds = np.zeros(Hq)
+    for h in range(Hq):
+        for i in range(n):
+            seen = [j for j in range(n) if 0 <= i - j and (window == 0 or i - j <= window - 1)]
+            Z = len(seen) + np.exp(s[h])
+            O_i = vs * sum(v[j, 0] for j in seen) / Z
+            D_i = float(dO[i, h] @ O_i)
+            for j in seen:
+                want_dv[j, 0] += vs * dO[i, h] / Z
+                # dq_i = s sum_j P_ij (v_scale <dO_i, v_j> - D_i) k_j
+                want_dq[i, h] += 0.5 / Z * (vs * float(dO[i, h] @ v[j, 0]) - D_i) * k[j, 0]
+            want_ds[h] -= np.exp(s[h]) / Z * D_i
+    np.testing.assert_allclose(dv, want_dv, atol=1e-13)
+    np.testing.assert_allclose(dq, want_dq, atol=1e-13)
+    np.testing.assert_allclose(ds, want_ds, atol=1e-13)
