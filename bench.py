@@ -73,6 +73,13 @@ def prefill_work(T, window):
     return flops, byts
 
 
+def varlen_prefill_work(lengths, window, out_bytes=2):
+    """prefill_work summed over a packed batch of sequences (one layer)."""
+    flops = sum(FLOP_PER_PAIR * HQ * visible_pairs(int(L), window) for L in lengths)
+    byts = int(sum(lengths)) * (HQ * DQK * 2 + HKV * (DQK + DV) * 2 + HQ * DV * out_bytes + HQ * 4)
+    return flops, byts
+
+
 def decode_work(lengths, window, capacity):
     ring = window > 0 and capacity == window
     vis = [min(L, capacity) if ring else (min(L, window) if window > 0 else L) for L in lengths]
@@ -111,6 +118,20 @@ def graph_us(fn, n=20, reps=10):
         ts.append(e0.elapsed_time(e1) / n)
     del g
     return 1e3 * float(np.median(ts[2:]))
+
+
+class L2Flush:
+    """Evicts the 126 MB L2 between timed launches: writes a 256 MB buffer, then
+    reads another, so the written (dirty) lines are written back to HBM during
+    the read, before the next timed event, and L2 is left holding clean lines."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
 
 
 def floor_s(flops, byts, peaks):
@@ -218,7 +239,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
         HQ, HKV, 64, W.DECODE_GA_CAPACITY, 0)), dtype=torch.uint8, device=dev)
     ws_sw = torch.empty(max(1, mimo.mimo_attn_decode_workspace_size(HQ, HKV, 64, SWA, SWA)),
                         dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # > 126 MB L2
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     def step(evs=None):
@@ -240,7 +261,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
     launches_per_step = 2 + (2 if ws_ga.numel() > 1 else 1) + (2 if ws_sw.numel() > 1 else 1)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     mimo.mimo_attn_device_status()
@@ -252,7 +273,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
     with ClockSampler(dev.index) as clk:
         t_wall = time.perf_counter()
         for k in range(args.steps):
-            flush.zero_()          # L2 flush between steps (outside the events)
+            flush()                # L2 flush between steps (outside the events)
             step(evs[k])
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -325,7 +346,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
                                                lse=l8, workspace=ws_ga)
         ms8 = []
         for i in range(args.warmup + 10):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
@@ -401,7 +422,7 @@ def run_ours(args, rank, world, peaks, peak_kind):
         dob = torch.randn(ob.shape, generator=gb, device=dev).to(ob.dtype)
         ms_b = []
         for i in range(args.warmup + 5):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             mimo.mimo_attn_prefill_backward(xb.q, xb.k, xb.v, ob, lb, dob, xb.sinks, 0,
@@ -423,6 +444,60 @@ def run_ours(args, rank, world, peaks, peak_kind):
                     "sink gradient in two small launches"}
         del xb, ob, lb, dob
 
+    # varlen 5:1 stack: 16 packed sequences, lengths ~U[512, 8192], six layers
+    # (windows 129 x 5, then global) with their own q/k/v and per-layer sinks
+    if extra is not None:
+        lengths5 = W.varlen_stack_lengths(0)
+        nt5, max5 = int(sum(lengths5)), int(max(lengths5))
+        sinks5 = W.stack_sinks(len(W.STACK_WINDOWS), seed=seed, device=dev)
+        layers = [W.prefill_inputs(lengths5, seed=seed + 30 + i, sinks=False, device=dev)
+                  for i in range(len(W.STACK_WINDOWS))]
+        outs5 = [torch.empty((nt5, HQ, DV), dtype=torch.bfloat16, device=dev) for _ in layers]
+        lses5 = [torch.empty((HQ, nt5), dtype=torch.float32, device=dev) for _ in layers]
+        nl = len(layers)
+        ms5 = []
+        for i in range(args.warmup + 5):
+            flush()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)]
+            ev[0].record(stream)
+            for li, (x, w) in enumerate(zip(layers, W.STACK_WINDOWS)):
+                mimo.mimo_attn_prefill(x.q, x.k, x.v, sinks5[li], w, x.cu_seqlens, max5,
+                                       out=outs5[li], lse=lses5[li])
+                ev[li + 1].record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ms5.append([ev[j].elapsed_time(ev[j + 1]) for j in range(nl)])
+        mimo.mimo_attn_device_status()
+        ms5 = np.array(ms5).mean(axis=0)
+        w5 = [varlen_prefill_work(lengths5, w) for w in W.STACK_WINDOWS]
+        f5 = [floor_s(f, b, peaks) for f, b in w5]
+        extra["prefill_varlen_stack_5to1_16seq"] = {
+            "ms": round(float(ms5.sum()), 4), "floor_ms": round(1e3 * sum(f5), 4),
+            "roofline_frac": round(1e3 * sum(f5) / float(ms5.sum()), 4),
+            "layers": [{"window": w, "ms": round(float(m), 4),
+                        "TFLOP/s": round(f / (m * 1e-3) / 1e12, 1),
+                        "GB/s": round(b / (m * 1e-3) / 1e9, 1),
+                        "roofline_frac": round(1e3 * fl / m, 4)}
+                       for w, m, (f, b), fl in zip(W.STACK_WINDOWS, ms5, w5, f5)],
+            "total_tokens": nt5, "useful_flop": int(sum(f for f, _ in w5)),
+            "algorithmic_bytes": int(sum(b for _, b in w5)), "launches": nl,
+            "note": "16 sequences, lengths default_rng(0).integers(512, 8193, 16), packed via "
+                    "cu_seqlens; layers 0-4 window 129, layer 5 global; bf16 out + lse; L2 "
+                    "flushed before each stack pass; floor = sum over layers of max(FLOP / "
+                    "tensor peak, bytes / HBM peak)"}
+        del layers, outs5, lses5
+        # the tiny sliding-window config (T=512, 16/1 heads, fp32 out): launch-bound
+        xt = W.prefill_inputs([512], hq=16, hkv=1, seed=seed + 40, device=dev)
+        ot = torch.empty((512, 16, DV), dtype=torch.float32, device=dev)
+        lt = torch.empty((16, 512), dtype=torch.float32, device=dev)
+        us_t = graph_us(lambda: mimo.mimo_attn_prefill(xt.q, xt.k, xt.v, xt.sinks, SWA,
+                                                       xt.cu_seqlens, 512, out=ot, lse=lt))
+        mimo.mimo_attn_device_status()
+        extra["prefill_tiny_swa_T512_H16"] = {
+            "us": round(us_t, 2), "launches": 1,
+            "note": "T=512, 16 query heads over 1 key/value head, window 129, fp32 out; device "
+                    "time per call (CUDA graph replay of 20 calls); launch/latency-bound"}
+
     res = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms, 4),
@@ -434,7 +509,9 @@ def run_ours(args, rank, world, peaks, peak_kind):
                                "(129-slot SWA ring)",
                    "heads_q": HQ, "heads_kv": HKV, "head_dim_qk": DQK, "head_dim_v": DV,
                    "seq_len": T_PREFILL, "decode_batch": 64, "parallelism": f"replicas{world}",
-                   "l2": "flushed between steps (256 MB write); every input > L2 except the "
+                   "l2": "flushed between steps (256 MB write, then a 256 MB read that "
+                         "writes the dirty lines back before the first event); every input > L2 "
+                         "except the "
                          "21 MB ring caches",
                    "floor_ms_per_step": round(floor_step_ms, 4),
                    "peaks": {**peaks, "source": peak_kind}},
@@ -658,14 +735,14 @@ def run_case(args):
             d = W.decode_inputs(lengths, cap, window, seed=3, device=dev)
             fn = lambda: mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, window, d.sinks)  # noqa: E731
             work = decode_work(lengths, window, cap)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         fn()
     torch.cuda.synchronize()
     ms = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         fn()

@@ -14,6 +14,7 @@ Entry points (same names as the C ABI):
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -39,6 +40,7 @@ EXPORTED = (
     "mimo_attn_decode",
     "mimo_attn_last_error",
     "mimo_attn_device_status",
+    "mimo_attn_set_device_status",
     "mimo_attn_decode_noalloc",
     "mimo_attn_decode_fp8_workspace_size",
     "mimo_attn_decode_fp8",
@@ -84,6 +86,8 @@ def _load():
     lib.mimo_attn_last_error.restype = ctypes.c_char_p
     lib.mimo_attn_device_status.argtypes = [vp]
     lib.mimo_attn_device_status.restype = i32
+    lib.mimo_attn_set_device_status.argtypes = [i32, vp]
+    lib.mimo_attn_set_device_status.restype = i32
     lib.mimo_attn_decode_fp8_workspace_size.argtypes = [dp, i32, i32, i32]
     lib.mimo_attn_decode_fp8_workspace_size.restype = sz
     lib.mimo_attn_decode_fp8.argtypes = [dp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, vp, vp, vp,
@@ -141,9 +145,31 @@ def _shape(t, shape, name):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def _stream(stream):
+def _same_device(dev, **tensors):
+    """Refuse tensors that live on another device than the call's (the library
+    launches on the current device and would dereference another GPU's memory)."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, but the call runs on {dev}")
+
+
+@contextlib.contextmanager
+def _on_device(dev):
+    """Make the tensors' device current for the call (launches, device queries)."""
+    if dev.type == "cuda":
+        with torch.cuda.device(dev):
+            yield
+    else:  # host tensors never reach the library: _ptr refuses them
+        yield
+
+
+def _stream(stream, dev):
+    """The stream to launch on: the caller's (which must belong to dev) or dev's
+    current stream."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
+    elif stream.device != dev:
+        raise ValueError(f"stream belongs to {stream.device}, but the call runs on {dev}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -174,12 +200,15 @@ def mimo_attn_prefill(q, k, v, sinks, window, cu_seqlens, max_seqlen, out=None, 
         out = torch.empty((nt, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((hq, nt), dtype=torch.float32, device=q.device)
+    dev = q.device
+    _same_device(dev, k=k, v=v, sinks=sinks, cu_seqlens=cu_seqlens, out=out, lse=lse)
     dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
-    _check(lib.mimo_attn_prefill(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16),
-                                 _ptr(v, "v", _BF16), _ptr(sinks, "sinks", _F32), int(window),
-                                 _ptr(cu_seqlens, "cu_seqlens", _I32), int(cu_seqlens.numel() - 1), nt,
-                                 int(max_seqlen), _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
-                                 _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_prefill(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16),
+                                     _ptr(v, "v", _BF16), _ptr(sinks, "sinks", _F32), int(window),
+                                     _ptr(cu_seqlens, "cu_seqlens", _I32), int(cu_seqlens.numel() - 1),
+                                     nt, int(max_seqlen), _ptr(out, "out", _OUT),
+                                     _ptr(lse, "lse", _F32), _stream(stream, dev)))
     return out, lse
 
 
@@ -216,16 +245,21 @@ def mimo_attn_decode(q, k_cache, v_cache, seqlens, window, sinks, out=None, lse=
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    dev = q.device
     dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
     need = int(lib.mimo_attn_decode_workspace_size(ctypes.byref(dims), B, C, int(window)))
     if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _same_device(dev, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens, sinks=sinks, out=out,
+                 lse=lse, workspace=workspace)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_cache, "k_cache", _BF16),
-                                _ptr(v_cache, "v_cache", _BF16), _ptr(seqlens, "seqlens", _I32), B, C,
-                                int(window), _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
-                                _ptr(lse, "lse", _F32), _ptr(workspace, "workspace"), wbytes,
-                                _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_decode(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                    _ptr(k_cache, "k_cache", _BF16), _ptr(v_cache, "v_cache", _BF16),
+                                    _ptr(seqlens, "seqlens", _I32), B, C, int(window),
+                                    _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                    _ptr(lse, "lse", _F32), _ptr(workspace, "workspace"), wbytes,
+                                    _stream(stream, dev)))
     return out, lse
 
 
@@ -249,17 +283,23 @@ def mimo_attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale_kv, seqlens, wind
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    dev = q.device
     dims = make_dims(hq, hkv, dqk, dv, softmax_scale, v_scale, out.dtype)
     need = int(lib.mimo_attn_decode_fp8_workspace_size(ctypes.byref(dims), B, C, int(window)))
     if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _same_device(dev, k_cache=k_cache, v_cache=v_cache, k_scale=k_scale, v_scale_kv=v_scale_kv,
+                 seqlens=seqlens, sinks=sinks, out=out, lse=lse, workspace=workspace)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.mimo_attn_decode_fp8(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_cache, "k_cache"),
-                                    _ptr(v_cache, "v_cache"), _ptr(k_scale, "k_scale", _F32),
-                                    _ptr(v_scale_kv, "v_scale_kv", _F32), _ptr(seqlens, "seqlens", _I32),
-                                    B, C, int(window), _ptr(sinks, "sinks", _F32),
-                                    _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
-                                    _ptr(workspace, "workspace"), wbytes, _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_decode_fp8(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                        _ptr(k_cache, "k_cache"), _ptr(v_cache, "v_cache"),
+                                        _ptr(k_scale, "k_scale", _F32),
+                                        _ptr(v_scale_kv, "v_scale_kv", _F32),
+                                        _ptr(seqlens, "seqlens", _I32), B, C, int(window),
+                                        _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                        _ptr(lse, "lse", _F32), _ptr(workspace, "workspace"), wbytes,
+                                        _stream(stream, dev)))
     return out, lse
 
 
@@ -272,12 +312,17 @@ def mimo_attn_rope_append(q, k_new, v_new, k_cache, v_cache, seqlens, window, ro
     _decode_shapes(q, k_cache, v_cache, seqlens, None, None, None)
     _shape(k_new, (B, hkv, dqk), "k_new")
     _shape(v_new, (B, hkv, v_cache.shape[3]), "v_new")
+    dev = q.device
+    _same_device(dev, k_new=k_new, v_new=v_new, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens)
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3])
     rd = dqk if rotary_dim is None else int(rotary_dim)
-    _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k_new, "k_new", _BF16),
-                                     _ptr(v_new, "v_new", _BF16), _ptr(k_cache, "k_cache", _BF16),
-                                     _ptr(v_cache, "v_cache", _BF16), _ptr(seqlens, "seqlens", _I32),
-                                     B, C, int(window), float(rope_theta), rd, _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_rope_append(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                         _ptr(k_new, "k_new", _BF16), _ptr(v_new, "v_new", _BF16),
+                                         _ptr(k_cache, "k_cache", _BF16),
+                                         _ptr(v_cache, "v_cache", _BF16),
+                                         _ptr(seqlens, "seqlens", _I32), B, C, int(window),
+                                         float(rope_theta), rd, _stream(stream, dev)))
     return q
 
 
@@ -294,10 +339,14 @@ def mimo_attn_decode_merge(part_out, part_lse, sinks, out=None, lse=None,
         out = torch.empty((B, hq, dv), dtype=out_dtype, device=part_out.device)
     if lse is None and return_lse:
         lse = torch.empty((B, hq), dtype=torch.float32, device=part_out.device)
+    dev = part_out.device
+    _same_device(dev, part_lse=part_lse, sinks=sinks, out=out, lse=lse)
     dims = make_dims(hq, 1, 192, dv, None, v_scale, out.dtype)
-    _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out, "part_out", _F32),
-                                      _ptr(part_lse, "part_lse", _F32), R, B, _ptr(sinks, "sinks", _F32),
-                                      _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32), _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_decode_merge(ctypes.byref(dims), _ptr(part_out, "part_out", _F32),
+                                          _ptr(part_lse, "part_lse", _F32), R, B,
+                                          _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                          _ptr(lse, "lse", _F32), _stream(stream, dev)))
     return out, lse
 
 
@@ -321,22 +370,45 @@ def mimo_attn_prefill_backward(q, k, v, out, lse, dout, sinks, window, cu_seqlen
     dk = torch.empty((nt, hkv, dqk), dtype=torch.float32, device=q.device)
     dv = torch.empty((nt, hkv, dv_dim), dtype=torch.float32, device=q.device)
     ds = None if sinks is None else torch.empty(hq, dtype=torch.float32, device=q.device)
+    dev = q.device
+    _same_device(dev, k=k, v=v, out=out, lse=lse, dout=dout, sinks=sinks, cu_seqlens=cu_seqlens)
     dims = make_dims(hq, hkv, dqk, dv_dim, softmax_scale, v_scale, out.dtype)
     need = int(lib.mimo_attn_prefill_backward_workspace_size(ctypes.byref(dims), nt))
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _check(lib.mimo_attn_prefill_backward(ctypes.byref(dims), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16),
-                                          _ptr(v, "v", _BF16), _ptr(out, "out", _OUT),
-                                          _ptr(lse, "lse", _F32), _ptr(dout, "dout", out.dtype),
-                                          _ptr(sinks, "sinks", _F32), int(window),
-                                          _ptr(cu_seqlens, "cu_seqlens", _I32), cu_seqlens.numel() - 1, nt,
-                                          int(max_seqlen), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds),
-                                          _ptr(ws), ws.numel(), _stream(stream)))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    with _on_device(dev):
+        _check(lib.mimo_attn_prefill_backward(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                              _ptr(k, "k", _BF16), _ptr(v, "v", _BF16),
+                                              _ptr(out, "out", _OUT), _ptr(lse, "lse", _F32),
+                                              _ptr(dout, "dout", out.dtype),
+                                              _ptr(sinks, "sinks", _F32), int(window),
+                                              _ptr(cu_seqlens, "cu_seqlens", _I32),
+                                              cu_seqlens.numel() - 1, nt, int(max_seqlen), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), _ptr(ds), _ptr(ws), ws.numel(),
+                                              _stream(stream, dev)))
     return dq, dk, dv, ds
 
 
-def mimo_attn_device_status(stream=None):
-    """Synchronise the stream; raise if a kernel recorded a device-side error."""
-    _check(lib.mimo_attn_device_status(_stream(stream)))
+def _current_device():
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def mimo_attn_device_status(stream=None, device=None):
+    """Synchronise the stream (default: the current stream of ``device``, itself
+    defaulting to the current device); raise if a kernel recorded a device-side
+    error on that device."""
+    dev = torch.device(device) if device is not None else (
+        stream.device if stream is not None else _current_device())
+    with _on_device(dev):
+        _check(lib.mimo_attn_device_status(_stream(stream, dev)))
+
+
+def mimo_attn_set_device_status(code, stream=None, device=None):
+    """Pre-load the device status word (test hook for the failure path; see
+    include/mimo_attn.h)."""
+    dev = torch.device(device) if device is not None else (
+        stream.device if stream is not None else _current_device())
+    with _on_device(dev):
+        _check(lib.mimo_attn_set_device_status(int(code), _stream(stream, dev)))
 
 
 def default_scale(dqk=192):
@@ -352,10 +424,15 @@ def mimo_attn_decode_noalloc(q, k_cache, v_cache, seqlens, window, sinks, out, l
     B, hq, dqk = q.shape
     C, hkv = k_cache.shape[1], k_cache.shape[2]
     _decode_shapes(q, k_cache, v_cache, seqlens, sinks, out, lse)
+    dev = q.device
+    _same_device(dev, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens, sinks=sinks, out=out,
+                 lse=lse)
     dims = make_dims(hq, hkv, dqk, v_cache.shape[3], softmax_scale, v_scale, out.dtype)
-    _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q, "q", _BF16),
-                                        _ptr(k_cache, "k_cache", _BF16), _ptr(v_cache, "v_cache", _BF16),
-                                        _ptr(seqlens, "seqlens", _I32), B, C, int(window),
-                                        _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
-                                        _ptr(lse, "lse", _F32), _stream(stream)))
+    with _on_device(dev):
+        _check(lib.mimo_attn_decode_noalloc(ctypes.byref(dims), _ptr(q, "q", _BF16),
+                                            _ptr(k_cache, "k_cache", _BF16),
+                                            _ptr(v_cache, "v_cache", _BF16),
+                                            _ptr(seqlens, "seqlens", _I32), B, C, int(window),
+                                            _ptr(sinks, "sinks", _F32), _ptr(out, "out", _OUT),
+                                            _ptr(lse, "lse", _F32), _stream(stream, dev)))
     return out, lse

@@ -55,7 +55,7 @@ struct BackwardParams {
   float* dsinks;             // [Hq] or null
   float* D;                  // [Hq, Nt] workspace
   float* psd;                // [Hq, Nt] workspace: exp(sigma - lse) * D
-  int total, Hq, Hkv, G, window, num_seqs;
+  int total, Hq, Hkv, G, window, num_seqs, max_seqlen;
   float scale, scale_log2, v_scale;
   int io_f32;                // out / dout are fp32
 };
@@ -190,6 +190,10 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_dq_kernel(const BackwardPar
 
   const int h = blockIdx.y, seq = blockIdx.z;
   const int b0 = p.cu_seqlens[seq], len = p.cu_seqlens[seq + 1] - b0;
+  if (!seq_in_bounds(b0, len, p.max_seqlen, p.total)) {  // bad cu_seqlens: touch nothing
+    if (threadIdx.x == 0) record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    return;
+  }
   const int nqt = (len + QR - 1) / QR;
   if ((int)blockIdx.x >= nqt) return;
   const int qt = nqt - 1 - (int)blockIdx.x;  // the longest key loops are issued first
@@ -355,6 +359,10 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_dkv_kernel(const BackwardPa
   // longest query loops are issued first.
   const int kt = (int)blockIdx.x / p.Hkv, g = (int)blockIdx.x % p.Hkv, seq = blockIdx.y;
   const int b0 = p.cu_seqlens[seq], len = p.cu_seqlens[seq + 1] - b0;
+  if (!seq_in_bounds(b0, len, p.max_seqlen, p.total)) {  // bad cu_seqlens: touch nothing
+    if (threadIdx.x == 0) record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    return;
+  }
   const int k0 = kt * kBwTile;
   if (k0 >= len) return;
   const int kv = min(kBwTile, len - k0);

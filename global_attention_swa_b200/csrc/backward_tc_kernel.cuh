@@ -72,6 +72,10 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   // key tiles in ascending order, KV heads fastest: the longest causal loops start first
   const int kt = (int)blockIdx.x / p.Hkv, g = (int)blockIdx.x % p.Hkv, seq = blockIdx.y;
   const int b0 = p.cu_seqlens[seq], len = p.cu_seqlens[seq + 1] - b0;
+  if (!seq_in_bounds(b0, len, p.max_seqlen, p.total)) {  // bad cu_seqlens: touch nothing
+    if (threadIdx.x == 0) record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    return;
+  }
   const int k0 = kt * kBtKeys;
   if (k0 >= len) return;  // the whole CTA, before any barrier or TMEM
   const int kv = min(kBtKeys, len - k0);

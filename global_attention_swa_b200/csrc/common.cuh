@@ -29,6 +29,15 @@ __device__ __forceinline__ bool timed_out_before() {
   return *reinterpret_cast<volatile int*>(&g_device_status) == 5 /* MIMO_ERR_TIMEOUT */;
 }
 
+// A packed sequence [b0, b0 + len) fits the call: it starts inside the token
+// range, its length is non-negative and at most max_seqlen, and it ends by
+// `total`.  The prefill and backward kernels check every sequence they touch
+// and skip (recording MIMO_ERR_INVALID_ARG) one that fails, so that a bad
+// cu_seqlens array cannot make them read or write outside the caller's buffers.
+__device__ __forceinline__ bool seq_in_bounds(int b0, int len, int max_seqlen, int total) {
+  return b0 >= 0 && len >= 0 && len <= max_seqlen && b0 <= total - len;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -389,6 +398,18 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
 // The two bf16 halves of a packed pair, as floats (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// The two f16 halves of a packed pair, as floats (exact).
+__device__ __forceinline__ float f16_lo(uint32_t u) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, l;\n\t}" : "=f"(r) : "r"(u));
+  return r;
+}
+__device__ __forceinline__ float f16_hi(uint32_t u) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.f32.f16 %0, h;\n\t}" : "=f"(r) : "r"(u));
+  return r;
+}
 
 // ---------------------------------------------------------------- mma.sync
 

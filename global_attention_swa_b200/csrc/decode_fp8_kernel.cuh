@@ -37,7 +37,7 @@ constexpr int kD8StageBytes = kD8KBytes + kD8VBytes;
 constexpr int kD8BoxBytes = kD8TileKeys * 64;  // 4096
 constexpr int kD8Threads = 160;                // 4 consumer warps + 1 producer warp
 constexpr int kD8SmemBytes = kD8Stages * kD8StageBytes + 1024 /*align*/ + 256 /*barriers*/;
-static_assert(4 * 16 * 128 * 4 + 2 * 4 * 16 * 4 <= kD8Stages * kD8StageBytes, "merge buffer fits");
+static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kD8Stages * kD8StageBytes, "merge buffer fits");
 
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
   return pack_f16(bf16_lo(u), bf16_hi(u));
@@ -72,7 +72,9 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
     fence_mbar_init();
   }
   __syncthreads();
-  const int ntiles = *abort_flag ? 0 : (nkeys + kD8TileKeys - 1) / kD8TileKeys;
+  // after a recorded timeout elsewhere, return at entry: nothing is read or written
+  if (*abort_flag) return;
+  const int ntiles = (nkeys + kD8TileKeys - 1) / kD8TileKeys;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -124,7 +126,8 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
 #pragma unroll
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY;
-    float l0 = 0.f, l1 = 0.f;
+    float l0 = 0.f, l1 = 0.f;              // per-thread partial sums (lse)
+    float lr0 = 0.f, lr1 = 0.f;            // the same over the rounded P (output normaliser)
 
     const int kw = warp * 16;
     // ldmatrix row of this lane: matrix m = lane / 8 covers keys kw + 8 (m & 1) + 0..7
@@ -190,6 +193,8 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
           pa[3] = pack_f16(p12, p13);
           l0 = l0 * a0 + ((p00 + p01) + (p10 + p11));
           l1 = l1 * a1 + ((p02 + p03) + (p12 + p13));
+          lr0 = lr0 * a0 + ((f16_lo(pa[0]) + f16_hi(pa[0])) + (f16_lo(pa[2]) + f16_hi(pa[2])));
+          lr1 = lr1 * a1 + ((f16_lo(pa[1]) + f16_hi(pa[1])) + (f16_lo(pa[3]) + f16_hi(pa[3])));
         }
         // rescale O only when some row's running max moved (2^0 is exactly 1)
         if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
@@ -238,10 +243,15 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    lr0 += __shfl_xor_sync(0xffffffffu, lr0, 1);
+    lr0 += __shfl_xor_sync(0xffffffffu, lr0, 2);
+    lr1 += __shfl_xor_sync(0xffffffffu, lr1, 1);
+    lr1 += __shfl_xor_sync(0xffffffffu, lr1, 2);
     asm volatile("bar.sync 1, 128;" ::: "memory");  // all consumers done with the stages
     float* so = reinterpret_cast<float*>(smem);      // [4 warps][16 rows][128]
     float* sm = so + 4 * 16 * 128;                   // [4][16] max
     float* sl = sm + 4 * 16;                         // [4][16] sum
+    float* slr = sl + 4 * 16;                        // [4][16] sum of the rounded P
     // o[4i + 2h] holds dims 32i + 16h + {4t, 4t+2} (even MMA), o[4i + 2h + 1]
     // dims 32i + 16h + {4t+1, 4t+3} (odd MMA), for rows r0 (c0, c1) and r0+8 (c2, c3).
 #pragma unroll
@@ -260,6 +270,8 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
       sm[warp * 16 + r0 + 8] = m1;
       sl[warp * 16 + r0] = l0;
       sl[warp * 16 + r0 + 8] = l1;
+      slr[warp * 16 + r0] = lr0;
+      slr[warp * 16 + r0 + 8] = lr1;
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     const int tid = threadIdx.x;
@@ -269,11 +281,12 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
 #pragma unroll
     for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 16 + row]);
     float wgt[4];
-    float Ls = 0.f;
+    float Ls = 0.f, Lrs = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       wgt[w] = (M == -INFINITY) ? 0.f : ex2(sm[w * 16 + row] - M);
       Ls += wgt[w] * sl[w * 16 + row];
+      Lrs += wgt[w] * slr[w * 16 + row];
     }
     float acc[16];
 #pragma unroll
@@ -288,12 +301,14 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
       if (p.nsplit == 1) {
         const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
         const float Mf = fmaxf(M, sg);
-        float scl = 0.f, Lf = 0.f;
+        float scl = 0.f, Lf = 0.f, Lrf = 0.f;
         if (Mf != -INFINITY) {
           scl = (M == -INFINITY) ? 0.f : ex2(M - Mf);
-          Lf = Ls * scl + ((sg == -INFINITY) ? 0.f : ex2(sg - Mf));
+          const float ps = (sg == -INFINITY) ? 0.f : ex2(sg - Mf);
+          Lf = Ls * scl + ps;
+          Lrf = Lrs * scl + ps;
         }
-        const float f = (Lf > 0.f) ? p.v_scale * p.kv_v_scale[g] * scl / Lf : 0.f;
+        const float f = (Lrf > 0.f) ? p.v_scale * p.kv_v_scale[g] * scl / Lrf : 0.f;
         const size_t ob = ((size_t)b * p.Hq + h) * 128 + c0;
         if (p.out_f32) {
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob);
@@ -321,8 +336,9 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
         for (int e = 0; e < 4; ++e)
           dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
         if ((tid & 7) == 0) {
-          p.ws_ml[(unit * 16 + row) * 2 + 0] = M;
-          p.ws_ml[(unit * 16 + row) * 2 + 1] = Ls;
+          p.ws_ml[(unit * 16 + row) * 4 + 0] = M;
+          p.ws_ml[(unit * 16 + row) * 4 + 1] = Ls;
+          p.ws_ml[(unit * 16 + row) * 4 + 2] = Lrs;
         }
       }
     }

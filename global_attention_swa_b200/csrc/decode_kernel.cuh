@@ -39,7 +39,7 @@ struct DecodeParams {
   void* out;               // [B, Hq, 128]
   float* lse;              // [B, Hq] or null
   float* ws_o;             // [B*Hkv*nsplit, 16, 128]
-  float* ws_ml;            // [B*Hkv*nsplit, 16, 2]
+  float* ws_ml;            // [B*Hkv*nsplit, 16, 4]: max, sum, sum of the rounded P, unused
   int B, C, Hq, Hkv, G;
   int window;
   int ring;     // 1: ring cache (C == window)
@@ -101,8 +101,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
-  // after a recorded timeout elsewhere, stream nothing (results are void anyway)
-  const int ntiles = *abort_flag ? 0 : (nkeys + kDecTileKeys - 1) / kDecTileKeys;
+  // after a recorded timeout elsewhere, return at entry: nothing is read or written
+  if (*abort_flag) return;
+  const int ntiles = (nkeys + kDecTileKeys - 1) / kDecTileKeys;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -149,7 +150,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY;  // running max (base 2) for rows r0, r0+8
-    float l0 = 0.f, l1 = 0.f;              // per-thread partial sums
+    float l0 = 0.f, l1 = 0.f;              // per-thread partial sums (lse)
+    float lr0 = 0.f, lr1 = 0.f;            // the same over the rounded P (output normaliser)
 
     const int kw = warp * 16;  // this warp's 16 keys within each tile
     const uint32_t sbase = smem_u32(smem);
@@ -212,6 +214,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           pa[3] = pack_bf16(p12, p13);
           l0 = l0 * a0 + ((p00 + p01) + (p10 + p11));
           l1 = l1 * a1 + ((p02 + p03) + (p12 + p13));
+          lr0 = lr0 * a0 + ((bf16_lo(pa[0]) + bf16_hi(pa[0])) + (bf16_lo(pa[2]) + bf16_hi(pa[2])));
+          lr1 = lr1 * a1 + ((bf16_lo(pa[1]) + bf16_hi(pa[1])) + (bf16_lo(pa[3]) + bf16_hi(pa[3])));
         }
         // rescale O only when some row's running max moved (2^0 is exactly 1)
         if (__any_sync(0xffffffffu, a0 != 1.f || a1 != 1.f)) {
@@ -252,10 +256,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    lr0 += __shfl_xor_sync(0xffffffffu, lr0, 1);
+    lr0 += __shfl_xor_sync(0xffffffffu, lr0, 2);
+    lr1 += __shfl_xor_sync(0xffffffffu, lr1, 1);
+    lr1 += __shfl_xor_sync(0xffffffffu, lr1, 2);
     asm volatile("bar.sync 1, 128;" ::: "memory");  // all consumers done with the stages
     float* so = reinterpret_cast<float*>(smem);      // [4 warps][16 rows][128]
     float* sm = so + 4 * 16 * 128;                   // [4][16] max
     float* sl = sm + 4 * 16;                         // [4][16] sum
+    float* slr = sl + 4 * 16;                        // [4][16] sum of the rounded P
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       const int col = n * 8 + cq;
@@ -269,6 +278,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       sm[warp * 16 + r0 + 8] = m1;
       sl[warp * 16 + r0] = l0;
       sl[warp * 16 + r0 + 8] = l1;
+      slr[warp * 16 + r0] = lr0;
+      slr[warp * 16 + r0 + 8] = lr1;
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     // 128 threads: thread -> (row = tid / 8, 16 columns)
@@ -279,11 +290,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
     for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 16 + row]);
     float wgt[4];
-    float Ls = 0.f;
+    float Ls = 0.f, Lrs = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       wgt[w] = (M == -INFINITY) ? 0.f : ex2(sm[w * 16 + row] - M);
       Ls += wgt[w] * sl[w * 16 + row];
+      Lrs += wgt[w] * slr[w * 16 + row];
     }
     float acc[16];
 #pragma unroll
@@ -299,12 +311,14 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         // fold the sink: it joins the normaliser only
         const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
         const float Mf = fmaxf(M, sg);
-        float scl = 0.f, Lf = 0.f;
+        float scl = 0.f, Lf = 0.f, Lrf = 0.f;
         if (Mf != -INFINITY) {
           scl = (M == -INFINITY) ? 0.f : ex2(M - Mf);
-          Lf = Ls * scl + ((sg == -INFINITY) ? 0.f : ex2(sg - Mf));
+          const float ps = (sg == -INFINITY) ? 0.f : ex2(sg - Mf);
+          Lf = Ls * scl + ps;
+          Lrf = Lrs * scl + ps;
         }
-        const float f = (Lf > 0.f) ? p.v_scale * scl / Lf : 0.f;
+        const float f = (Lrf > 0.f) ? p.v_scale * scl / Lrf : 0.f;
         const size_t ob = ((size_t)b * p.Hq + h) * 128 + c0;
         if (p.out_f32) {
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob);
@@ -332,8 +346,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         for (int e = 0; e < 4; ++e)
           dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
         if ((tid & 7) == 0) {
-          p.ws_ml[(unit * 16 + row) * 2 + 0] = M;
-          p.ws_ml[(unit * 16 + row) * 2 + 1] = Ls;
+          p.ws_ml[(unit * 16 + row) * 4 + 0] = M;
+          p.ws_ml[(unit * 16 + row) * 4 + 1] = Ls;
+          p.ws_ml[(unit * 16 + row) * 4 + 2] = Lrs;
         }
       }
     }
@@ -342,14 +357,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
 // Merge the split partials of every (b, query head) and fold the sink:
 //   M = max(sigma, max_c m_c),  Z = 2^(sigma-M) + sum_c 2^(m_c-M) l_c,
-//   out = v_scale * sum_c 2^(m_c-M) o_c / Z,   lse = ln Z + M ln 2
+//   out = v_scale * sum_c 2^(m_c-M) o_c / Z~,   lse = ln Z + M ln 2
+// where Z~ is Z over the splits' sums of the rounded P (the values their P.V used)
 // (times the V scale of the KV head for FP8 caches, whose partials are in code units).
 // One warp per (b, h); lane handles 4 of the 128 value columns.
 __global__ void __launch_bounds__(256)
     decode_combine_kernel(const DecodeParams p) {
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= p.B * p.Hq) return;
+  if (wid >= p.B * p.Hq || timed_out_before()) return;  // after a recorded timeout: write nothing
   const int b = wid / p.Hq, h = wid % p.Hq;
   const int g = h / p.G, row = h % p.G;
   int lo, hi;
@@ -358,16 +374,18 @@ __global__ void __launch_bounds__(256)
   const size_t unit0 = ((size_t)b * p.Hkv + g) * p.nsplit;
   const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
   float M = sg;
-  for (int c = 0; c < nused; ++c) M = fmaxf(M, p.ws_ml[((unit0 + c) * 16 + row) * 2]);
+  for (int c = 0; c < nused; ++c) M = fmaxf(M, p.ws_ml[((unit0 + c) * 16 + row) * 4]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float Z = 0.f;
+  float Z = 0.f, Zr = 0.f;
   if (M != -INFINITY) {
     Z = (sg == -INFINITY) ? 0.f : ex2(sg - M);
+    Zr = Z;
     for (int c = 0; c < nused; ++c) {
-      const float mc = p.ws_ml[((unit0 + c) * 16 + row) * 2];
-      const float lc = p.ws_ml[((unit0 + c) * 16 + row) * 2 + 1];
+      const float4 ml = *reinterpret_cast<const float4*>(p.ws_ml + ((unit0 + c) * 16 + row) * 4);
+      const float mc = ml.x;
       const float w = (mc == -INFINITY) ? 0.f : ex2(mc - M);
-      Z += w * lc;
+      Z += w * ml.y;
+      Zr += w * ml.z;
       const float4 oc = reinterpret_cast<const float4*>(p.ws_o + ((unit0 + c) * 16 + row) * 128)[lane];
       acc.x += w * oc.x;
       acc.y += w * oc.y;
@@ -376,7 +394,7 @@ __global__ void __launch_bounds__(256)
     }
   }
   const float vs = p.kv_v_scale ? p.kv_v_scale[g] : 1.f;
-  const float f = (Z > 0.f) ? p.v_scale * vs / Z : 0.f;
+  const float f = (Zr > 0.f) ? p.v_scale * vs / Zr : 0.f;
   const size_t ob = ((size_t)b * p.Hq + h) * 128 + lane * 4;
   if (p.out_f32) {
     *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob) =

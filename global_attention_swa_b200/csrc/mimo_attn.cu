@@ -233,7 +233,8 @@ DecodePlan decode_plan(int batch, int hkv, int capacity, int window) {
 size_t workspace_bytes_of(int batch, int hkv, const DecodePlan& pl) {
   if (pl.nsplit <= 1) return 0;
   const size_t units = (size_t)batch * hkv * pl.nsplit;
-  return units * 16 * 128 * sizeof(float) + units * 16 * 2 * sizeof(float);
+  // partial O [units][16][128], then (max, sum, rounded-P sum, unused) [units][16][4]
+  return units * 16 * 128 * sizeof(float) + units * 16 * 4 * sizeof(float);
 }
 
 }  // namespace
@@ -300,6 +301,7 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
     sp.N = Nsw;
     sp.window = window;
     sp.num_seqs = num_seqs;
+    sp.max_seqlen = max_seqlen;
     sp.num_pairs = (max_seqlen + 2 * QB - 1) / (2 * QB);
     const long items = (long)sp.num_pairs * Hkv * num_seqs;
     if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
@@ -350,6 +352,7 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
   p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
   p.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
   p.num_seqs = num_seqs;
+  p.max_seqlen = max_seqlen;
   p.num_qtiles = (max_seqlen + mimo::kPfTile - 1) / mimo::kPfTile;
   const long items = (long)p.num_qtiles * Hkv * p.pairs_per_group * num_seqs;
   if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
@@ -634,6 +637,7 @@ mimo_status_t mimo_attn_prefill_backward(const mimo_attn_dims_t* dims, const voi
   p.G = p.Hq / p.Hkv;
   p.window = window;
   p.num_seqs = num_seqs;
+  p.max_seqlen = max_seqlen;
   p.scale = dims->softmax_scale > 0.f ? dims->softmax_scale : 1.0f / std::sqrt((float)dims->head_dim_qk);
   p.scale_log2 = scale_log2_of(dims);
   p.v_scale = v_scale_of(dims);
@@ -704,6 +708,18 @@ mimo_status_t mimo_attn_device_status(void* stream) {
     return st;
   if (v == 0) return ok();
   return fail(static_cast<mimo_status_t>(v), "device status %d recorded by a kernel", v);
+}
+
+mimo_status_t mimo_attn_set_device_status(int code, void* stream) {
+  if (code < MIMO_OK || code > MIMO_ERR_TIMEOUT)
+    return fail(MIMO_ERR_INVALID_ARG, "status code %d is not a mimo_status_t", code);
+  // pageable source: the value is captured before the call returns
+  mimo_status_t st;
+  if ((st = cuda_check(cudaMemcpyToSymbolAsync(mimo::g_device_status, &code, sizeof(int), 0,
+                                               cudaMemcpyHostToDevice, (cudaStream_t)stream),
+                       "write status")))
+    return st;
+  return ok();
 }
 
 }  // extern "C"

@@ -68,6 +68,7 @@ struct PrefillParams {
   int window;
   int pairs_per_group;        // ceil(G / 2)
   int num_seqs;
+  int max_seqlen;
   int num_qtiles;             // ceil(max_seqlen / 128)
   int num_items;              // num_qtiles * Hkv * pairs_per_group * num_seqs
   float scale_log2;           // softmax_scale * log2(e)
@@ -111,6 +112,12 @@ __device__ __forceinline__ PfItem pf_decode(const PrefillParams& p, int item) {
   it.len = p.cu_seqlens[seq + 1] - it.b0;
   it.q0 = qt * kPfTile;
   it.valid = it.q0 < it.len;
+  if (!seq_in_bounds(it.b0, it.len, p.max_seqlen, p.total)) {
+    // a cu_seqlens entry out of order or past total_tokens, or a sequence
+    // longer than max_seqlen: no row of it is read or written
+    record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    it.valid = false;
+  }
   if (it.valid) {
     const int last_q = min(it.q0 + kPfTile - 1, it.len - 1);
     const int j_hi = last_q / kPfTile;
@@ -330,7 +337,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int qpos = it.q0 + r;
       const float sg2 = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
       float m = sg2;
-      float l = p.sinks ? 1.f : 0.f;
+      float l = p.sinks ? 1.f : 0.f;   // exact row sum (lse)
+      float lr = l;                    // sum of the bf16-rounded P that enter P.V (output)
       for (int t = 0; t < it.n_kt; ++t, ++tg) {
         const int kpos0 = (it.j_lo + t) * kPfTile;
         if (!(ok = wait_bounded(&s_full[i], tg & 1, abort_flag))) break;
@@ -364,16 +372,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (m_new - m > kRescaleLog2) {  // false when both are -inf (NaN compare)
           alpha = ex2(m - m_new);
           l *= alpha;
+          lr *= alpha;
           m = m_new;
           rescale_o = (t > 0);
         }
         const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        // P = 2^(s*scale - m), rounded to bf16 for the PV product; the row sum
-        // keeps the unrounded values so that lse stays exact to fp32.
+        // P = 2^(s*scale - m), rounded to bf16 for the PV product.  Two row sums:
+        // the unrounded values (lse, exact to fp32) and the rounded ones, which
+        // normalise the output, so that out = sum_j P~_j v_j / (sum_j P~_j + sink)
+        // weights the value rows by exactly the P that multiplied them.
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float2 nm2 = make_float2(neg_m, neg_m);
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                         make_float2(0.f, 0.f)};
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 acr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -382,13 +393,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float2 x = fma2(make_float2(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]), sc2, nm2);
             const float2 e = make_float2(ex2(x.x), ex2(x.y));
             pk[c] = pack_bf16(e.x, e.y);
-            acc[c & 3] = add2(acc[c & 3], e);
+            acc[c & 1] = add2(acc[c & 1], e);
+            acr[c & 1] = add2(acr[c & 1], make_float2(bf16_lo(pk[c]), bf16_hi(pk[c])));
           }
           tmem_st32(tS + 32 * half, pk);
         }
-        const float2 a01 = add2(acc[0], acc[1]), a23 = add2(acc[2], acc[3]);
-        const float2 a = add2(a01, a23);
+        const float2 a = add2(acc[0], acc[1]), ar = add2(acr[0], acr[1]);
         l += a.x + a.y;
+        lr += ar.x + ar.y;
         // O of the previous tile is complete here: S_i(t) was committed after PV_i(t-1).
         if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
@@ -417,7 +429,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ++n;
       if (qpos < it.len) {
         const int tok = it.b0 + qpos;
-        const float f = (l > 0.f) ? p.v_scale / l : 0.f;
+        const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
         const size_t ob = ((size_t)tok * p.Hq + h) * 128;
         if (p.out_f32) {
           float* dst = reinterpret_cast<float*>(p.out) + ob;

@@ -50,7 +50,7 @@ struct SwaParams {
   void* out;
   float* lse;
   int total, Hq, Hkv, G, QB, N, window;
-  int num_seqs, num_pairs, num_items;   // items = pairs of blocks
+  int num_seqs, max_seqlen, num_pairs, num_items;   // items = pairs of blocks
   float scale_log2, v_scale;
   int out_f32, out_v8;
 };
@@ -72,6 +72,12 @@ __device__ __forceinline__ SwItem sw_decode(const SwaParams& p, int item) {
   it.len = p.cu_seqlens[seq + 1] - it.b0;
   it.q0 = qb * 2 * p.QB;
   it.valid = it.q0 < it.len;
+  if (!seq_in_bounds(it.b0, it.len, p.max_seqlen, p.total)) {
+    // a cu_seqlens entry out of order or past total_tokens, or a sequence
+    // longer than max_seqlen: no row of it is read or written
+    record_status(1 /* MIMO_ERR_INVALID_ARG */);
+    it.valid = false;
+  }
   it.nblk = (it.q0 + p.QB < it.len) ? 2 : 1;
   return it;
 }
@@ -108,7 +114,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   uint64_t* ml_empty = bars + 16; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
-  float2* ml = reinterpret_cast<float2*>(smem + kSwOffML);  // [2][128] (m, l) per row
+  float2* ml = reinterpret_cast<float2*>(smem + kSwOffML);  // [2][128] (output factor, lse) per row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 12) {
@@ -296,8 +302,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       }
       const float m = fmaxf(sg2, fmaxf(mx0, mx1) * p.scale_log2);
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same columns
-      float l0 = 0.f, l1 = 0.f;
+      // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same
+      // columns.  The unrounded sum gives lse; the sum of the rounded P (the
+      // values P.V multiplies) normalises the output.
+      float2 l2 = make_float2(0.f, 0.f), lr2 = make_float2(0.f, 0.f);
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t v[16], pk[8];
         tmem_load16_sync(tS + c0, v);
@@ -306,10 +314,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           for (int e = 0; e < 8; ++e) {
             const float2 x = fma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
                                   make_float2(p.scale_log2, p.scale_log2), make_float2(neg_m, neg_m));
-            const float p0 = ex2(x.x), p1 = ex2(x.y);
-            l0 += p0;
-            l1 += p1;
-            pk[e] = pack_bf16(p0, p1);
+            const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+            pk[e] = pack_bf16(pe.x, pe.y);
+            l2 = add2(l2, pe);
+            lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
           }
         } else {
 #pragma unroll
@@ -317,11 +325,11 @@ __global__ void __launch_bounds__(kSwThreads, 1)
             const int c = c0 + 2 * e;
             const float x0 = fmaf(__uint_as_float(v[2 * e]), p.scale_log2, neg_m);
             const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, neg_m);
-            const float p0 = (c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f;
-            const float p1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f;
-            l0 += p0;
-            l1 += p1;
-            pk[e] = pack_bf16(p0, p1);
+            const float2 pe = make_float2((c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f,
+                                          (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f);
+            pk[e] = pack_bf16(pe.x, pe.y);
+            l2 = add2(l2, pe);
+            lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
           }
         }
         tmem_st8(tS + c0 / 2, pk);
@@ -329,10 +337,16 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
-      float l = l0 + l1;
-      if (p.sinks && m != -INFINITY) l += ex2(sg2 - m);
+      float l = l2.x + l2.y, lr = lr2.x + lr2.y;
+      if (p.sinks && m != -INFINITY) {
+        const float ps = ex2(sg2 - m);
+        l += ps;
+        lr += ps;
+      }
+      const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
+      const float lse = (l > 0.f) ? (m * 0.6931471805599453f + logf(l)) : -INFINITY;
       if (n >= 2 && !(ok = wait_bounded(&ml_empty[b], ((n >> 1) - 1) & 1, abort_flag))) break;
-      ml[b * 128 + r] = make_float2(m, l);
+      ml[b * 128 + r] = make_float2(f, lse);
       mbar_arrive(&ml_full[b]);
     }
   } else if (warp < 12) {
@@ -356,8 +370,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       const bool live = qpos < it.len;
       const int tok = it.b0 + qpos;
       const int hg = it.g * p.G + hh;
-      const float l = mlv.y;
-      const float f = (l > 0.f) ? p.v_scale / l : 0.f;
+      const float f = mlv.x;
       const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
       // O in two 64-column halves (registers: 448 threads leave 128 per thread);
       // O is released to the next P.V after the second half is in registers.
@@ -411,11 +424,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           }
         }
       }
-      if (live) {
-        if (p.lse)
-          p.lse[(size_t)hg * p.total + tok] =
-              (l > 0.f) ? (mlv.x * 0.6931471805599453f + logf(l)) : -INFINITY;
-      }
+      if (live && p.lse) p.lse[(size_t)hg * p.total + tok] = mlv.y;
     }
   }
 

@@ -298,7 +298,10 @@ mimo_status_t mimo_attn_decode_fp8(const mimo_attn_dims_t* dims, const void* q,
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the previous call's
+ * capture.  The cached address belongs to the device's context as it was at
+ * that first call: after cudaDeviceReset (or anything else that destroys the
+ * device's primary context) do not call this entry point again on that device
+ * in the same process.  All calls share the one array and it keeps the previous call's
  * contents (nothing in it needs to start at zero): calls that overlap on the
  * GPU, on any streams, race and corrupt each other's results.
  */
@@ -317,6 +320,18 @@ const char* mimo_attn_last_error(void);
  * MIMO_OK, MIMO_ERR_TIMEOUT, MIMO_ERR_INVALID_ARG or MIMO_ERR_CUDA.
  */
 mimo_status_t mimo_attn_device_status(void* stream);
+
+/*
+ * Writes `code` (a mimo_status_t value) into the device status word,
+ * ordered on `stream`: kernels launched on it afterwards see the new value.
+ * A diagnostic hook for testing the failure path without a failing GPU.
+ * With MIMO_ERR_TIMEOUT pre-loaded, every kernel that has bounded waits
+ * (prefill, decode, FP8 decode, the decode combine, the tcgen05 backward)
+ * returns at entry, as it does after a real timed-out wait elsewhere, and
+ * writes none of its outputs.  mimo_attn_device_status() then reports the
+ * code and clears it.  Codes outside 0..5 return MIMO_ERR_INVALID_ARG.
+ */
+mimo_status_t mimo_attn_set_device_status(int code, void* stream);
 
 #ifdef __cplusplus
 }

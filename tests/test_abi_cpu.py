@@ -232,7 +232,7 @@ def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
 
     monkeypatch.setattr(mimo, "lib", FakeLib())
     monkeypatch.setattr(mimo, "_ptr", host_ptr)
-    monkeypatch.setattr(mimo, "_stream", lambda stream: None)
+    monkeypatch.setattr(mimo, "_stream", lambda stream, dev: None)
     bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
     B, C, Hq, Hkv, Nt = 2, 16, 4, 1, 24
     q = torch.zeros((Nt, Hq, 192), dtype=bf)
@@ -263,6 +263,7 @@ def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
                                kc, vc, sl, 16, 10000.0)
     mimo.mimo_attn_decode_merge(torch.zeros((3, B, Hq, 128)), torch.zeros((3, B, Hq)), sinks)
     mimo.mimo_attn_decode_noalloc(qd, kc, vc, sl, 0, sinks, torch.zeros((B, Hq, 128), dtype=bf))
+    seen = list(calls)
     with pytest.raises(TypeError, match="seqlens"):
         mimo.mimo_attn_decode(qd, kc, vc, sl.long(), 0, sinks)
     # sizes that disagree with the ones derived from q would be read past their end
@@ -278,5 +279,51 @@ def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
         mimo.mimo_attn_decode_merge(torch.zeros((3, B, Hq, 128)), torch.zeros((2, B, Hq)), sinks)
     with pytest.raises(ValueError, match="contiguous"):
         mimo.mimo_attn_decode(qd, kc[:, ::2], vc[:, ::2], sl, 0, sinks)
+    # every tensor must be on the call's device (q's): the library launches on one
+    # device and would dereference another GPU's addresses
+    calls.clear()
+    meta = lambda t: t.to("meta")  # noqa: E731  (a device other than q's)
+    with pytest.raises(ValueError, match="v is on meta"):
+        mimo.mimo_attn_prefill(q, k, meta(v), sinks, 0, cu, 14)
+    with pytest.raises(ValueError, match="cu_seqlens is on meta"):
+        mimo.mimo_attn_prefill(q, k, v, sinks, 0, meta(cu), 14)
+    with pytest.raises(ValueError, match="out is on meta"):
+        mimo.mimo_attn_prefill(q, k, v, sinks, 0, cu, 14, out=torch.empty((Nt, Hq, 128), device="meta"))
+    with pytest.raises(ValueError, match="k_cache is on meta"):
+        mimo.mimo_attn_decode(qd, meta(kc), vc, sl, 0, sinks)
+    with pytest.raises(ValueError, match="workspace is on meta"):
+        mimo.mimo_attn_decode(qd, kc, vc, sl, 0, sinks, workspace=torch.empty(16, device="meta"))
+    with pytest.raises(ValueError, match="k_scale is on meta"):
+        mimo.mimo_attn_decode_fp8(qd, codes_k, codes_v, meta(scale), scale, sl, 0, sinks)
+    with pytest.raises(ValueError, match="v_cache is on meta"):
+        mimo.mimo_attn_rope_append(qd, torch.zeros((B, Hkv, 192), dtype=bf),
+                                   torch.zeros((B, Hkv, 128), dtype=bf), kc, meta(vc), sl, 16, 1e4)
+    with pytest.raises(ValueError, match="sinks is on meta"):
+        mimo.mimo_attn_decode_merge(torch.zeros((3, B, Hq, 128)), torch.zeros((3, B, Hq)), meta(sinks))
+    with pytest.raises(ValueError, match="dout is on meta"):
+        mimo.mimo_attn_prefill_backward(q, k, v, out, lse, meta(torch.zeros_like(out)), sinks, 0, cu, 14)
+    with pytest.raises(ValueError, match="seqlens is on meta"):
+        mimo.mimo_attn_decode_noalloc(qd, kc, vc, meta(sl), 0, sinks, torch.zeros((B, Hq, 128), dtype=bf))
+    # refused before any entry point that touches the device (size queries are host-only)
+    assert [c for c in calls if not c.endswith("_workspace_size")] == []
     assert {"mimo_attn_prefill", "mimo_attn_prefill_backward", "mimo_attn_decode", "mimo_attn_decode_fp8",
-            "mimo_attn_rope_append", "mimo_attn_decode_merge", "mimo_attn_decode_noalloc"} <= set(calls)
+            "mimo_attn_rope_append", "mimo_attn_decode_merge", "mimo_attn_decode_noalloc"} <= set(seen)
+
+
+def test_binding_refuses_a_stream_of_another_device():
+    """A caller's stream must belong to the device the tensors live on."""
+    import types
+
+    import torch
+
+    other = types.SimpleNamespace(device=torch.device("cuda", 1), cuda_stream=0)
+    with pytest.raises(ValueError, match="stream belongs to cuda:1"):
+        mimo._stream(other, torch.device("cuda", 0))
+    same = types.SimpleNamespace(device=torch.device("cuda", 0), cuda_stream=1234)
+    assert mimo._stream(same, torch.device("cuda", 0)).value == 1234
+
+
+def test_set_device_status_rejects_codes_outside_the_enum():
+    assert mimo.lib.mimo_attn_set_device_status(6, None) == mimo.MIMO_ERR_INVALID_ARG
+    assert mimo.lib.mimo_attn_set_device_status(-1, None) == mimo.MIMO_ERR_INVALID_ARG
+    assert "status code" in mimo.lib.mimo_attn_last_error().decode()

@@ -63,3 +63,17 @@ def test_decode_work_at_the_benchmark_sizes():
     # e4m3 caches: one byte per element plus the per-KV-head K and V scales
     _, b8 = bench.decode_fp8_work(lengths, 0, W.DECODE_GA_CAPACITY)
     assert b8 == total * 1280 + 64 * 64 * (192 * 2 + 128 * 2 + 4) + 2 * 4 * 4
+
+
+def test_varlen_stack_work():
+    """Config 5: 16 packed sequences ~U[512, 8192] (Nt = 70,172), five window-129
+    layers and one global layer: per-layer work is the sum over sequences."""
+    lengths = W.varlen_stack_lengths(0)
+    assert len(lengths) == 16 and sum(lengths) == 70172
+    f_swa, b_swa = bench.varlen_prefill_work(lengths, 129)
+    f_ga, b_ga = bench.varlen_prefill_work(lengths, 0)
+    assert f_swa == 640 * 64 * sum(brute_pairs(L, 129) for L in lengths[:2]) + 640 * 64 * sum(
+        bench.visible_pairs(L, 129) for L in lengths[2:])
+    assert f_ga == 640 * 64 * sum(L * (L + 1) // 2 for L in lengths)
+    assert b_swa == b_ga == 70172 * 43_776
+    assert round((5 * f_swa + f_ga) / 1e12, 2) == 9.99

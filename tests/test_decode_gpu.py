@@ -47,7 +47,7 @@ def test_model_heads_bf16_out():
     x = W.decode_inputs([3000, 17, 4097], 8192, 0, seed=9)
     out, lse = run(x, torch.bfloat16)
     ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, 0, x.sinks)
-    P.strict(out, ro, lse, rl, what="64/4 heads")
+    P.check(out, ro, lse, rl, what="64/4 heads")
 
 
 def test_split_count_does_not_change_the_result():
@@ -65,7 +65,7 @@ def test_split_count_does_not_change_the_result():
         outs.append(run(x)[0])
     ro, _ = oracle.decode(a.q, a.k_cache, a.v_cache, a.seqlens, 0, a.sinks)
     for o in outs:
-        P.strict(o, ro, what="split plan")
+        P.check(o, ro, what="split plan")
 
 
 def test_decode_equals_last_prefill_row():
@@ -104,7 +104,7 @@ def test_ring_matches_linear_window():
     assert (a - b).abs().max().item() < 2e-3
     assert (la - lb).abs().max().item() < 1e-4
     ro, rl = oracle.decode(x.q[L - 1:L], x.k[None], x.v[None], [L], 129, x.sinks, ring=False)
-    P.strict(a, ro, la, rl, what="ring")
+    P.check(a, ro, la, rl, what="ring")
 
 
 def test_full_size_decode_global_and_ring():
@@ -118,11 +118,11 @@ def test_full_size_decode_global_and_ring():
     pick = sorted({int(np.argmax(Ls)), int(np.argmin(Ls)), 0, 17, 63})
     ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, 0, x.sinks, batch_index=pick)
     idx = torch.as_tensor(pick, device="cuda")
-    P.strict(out[idx], ro, lse[idx], rl, what="GA decode b64")
+    P.check(out[idx], ro, lse[idx], rl, what="GA decode b64")
     del x
     torch.cuda.empty_cache()
     r = W.decode_inputs(lengths, 129, 129, seed=1, device="cuda")
     out, lse = mimo.mimo_attn_decode(r.q, r.k_cache, r.v_cache, r.seqlens, 129, r.sinks)
     mimo.mimo_attn_device_status()
     ro, rl = oracle.decode(r.q, r.k_cache, r.v_cache, r.seqlens, 129, r.sinks)
-    P.strict(out, ro, lse, rl, what="SWA ring decode b64")
+    P.check(out, ro, lse, rl, what="SWA ring decode b64")
