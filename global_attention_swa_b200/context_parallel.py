@@ -50,9 +50,10 @@ def context_parallel_decode(q, k_cache, v_cache, part_lens, sinks, group=None,
     merge = merge or _merge_cuda
     part_out, part_lse = local_part(q, k_cache, v_cache, part_lens, softmax_scale)
     B, hq, dv = part_out.shape
-    # one exchange: each rank's (out, lse) packed as [B, Hq, Dv + 1] fp32 (the merge
-    # takes fp32 parts; lse rounded to a 16-bit type would shift the merge weights)
-    packed = torch.cat([part_out.reshape(B, hq, dv).float(), part_lse.reshape(B, hq, 1).float()],
+    # one exchange: each rank's (out, lse) packed as [B, Hq, Dv + 1], in fp32 at least
+    # (lse rounded to a 16-bit type would shift the merge weights)
+    dt = torch.promote_types(torch.promote_types(part_out.dtype, part_lse.dtype), torch.float32)
+    packed = torch.cat([part_out.reshape(B, hq, dv).to(dt), part_lse.reshape(B, hq, 1).to(dt)],
                        dim=2).contiguous()
     world = dist.get_world_size(group)
     gathered = [torch.empty_like(packed) for _ in range(world)]
