@@ -439,9 +439,9 @@ def run_ours(args, rank, world, peaks, peak_kind):
             "ms": round(m_b, 3), "TFLOP/s": round(fb / (m_b * 1e-3) / 1e12, 1),
             "roofline_frac": round(fb / (m_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
             "bound": "tensor", "useful_flop": fb, "launches": 4,
-            "note": "dq, dk, dv, dsinks (the forward's out and lse as inputs): dK and dV in one "
-                    "tcgen05 pass, dQ with warp-level mma.sync (recomputing S and dP), D and the "
-                    "sink gradient in two small launches"}
+            "note": "dq, dk, dv, dsinks (the forward's out and lse as inputs): dQ in one tcgen05 "
+                    "pass over 128-key tiles, dK and dV in another (each recomputes S and dP), D "
+                    "and the sink gradient in two small launches"}
         del xb, ob, lb, dob
 
     # varlen 5:1 stack: 16 packed sequences, lengths ~U[512, 8192], six layers

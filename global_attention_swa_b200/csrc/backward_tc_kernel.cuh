@@ -25,6 +25,11 @@
 // TMEM columns: dV [0,128)  dK [128,320)  S^T_0 [320,384)  dP^T [384,448)
 // S^T_1 [448,512).  The next item's S^T goes to the other buffer while the
 // softmax works on the current one; its dP^T follows the current dK product.
+// The softmax hands its results over in two steps: P^T (the dV product can
+// start) and then dS^T (the dK product), so the exponentials of one item
+// overlap the dK and next dP^T products of the item before.  Masking is per
+// key row as a range of visible query columns: one warp-uniform branch per
+// item (all visible / some masked), selects inside.
 //
 // Every wait is bounded (1 s of %globaltimer); a wait that gives up records
 // MIMO_ERR_TIMEOUT and the CTA unwinds, freeing its TMEM.
@@ -48,8 +53,29 @@ constexpr int kBtStages = 3;
 constexpr int kBtOffStage = kBtOffV + kBtVBytes;
 constexpr int kBtOffLD = kBtOffStage + kBtStages * kBtStage;  // 2 x {lse log2e [64], D [64]}
 constexpr int kBtOffBar = kBtOffLD + 2 * 2 * kBtQ * 4;
-constexpr int kBtSmemBytes = kBtOffBar + 128 + 1024;      // barriers + alignment slack
+constexpr int kBtSmemBytes = kBtOffBar + 256 + 1024;      // barriers + alignment slack
 constexpr uint32_t kBtColDV = 0, kBtColDK = 128, kBtColS0 = 320, kBtColDP = 384, kBtColS1 = 448;
+
+// P^T row of one item: P = 2^(S s log2e - lse log2e) for the 64 query columns
+// (lse log2e in ld4[0..15]), zero outside [c_lo, c_hi] when kMasked (selects,
+// no branches); also packed to bf16 pairs for the dV product.
+template <bool kMasked>
+__device__ __forceinline__ void bwd_p_tile(float (&pe)[64], const float4* ld4, float scale_log2,
+                                           int c_lo, int c_hi, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c4 = 0; c4 < 16; ++c4) {
+    const float4 l4 = ld4[c4];
+    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int qc = 4 * c4 + e;
+      const float x = ex2(fmaf(pe[qc], scale_log2, -lv[e]));
+      pe[qc] = (!kMasked || (qc >= c_lo && qc <= c_hi)) ? x : 0.f;
+    }
+    pk[2 * c4] = pack_bf16(pe[4 * c4], pe[4 * c4 + 1]);
+    pk[2 * c4 + 1] = pack_bf16(pe[4 * c4 + 2], pe[4 * c4 + 3]);
+  }
+}
 
 __global__ void __launch_bounds__(kBtThreads, 1)
     bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -61,12 +87,14 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;   // [kBtStages]
   uint64_t* q_empty = bars + 4;  // [kBtStages]
-  uint64_t* s_full = bars + 7;
-  uint64_t* p_full = bars + 8;
-  uint64_t* ld_full = bars + 9;  // [2]
-  uint64_t* done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+  uint64_t* s_full = bars + 7;    // [2] S^T of items with j & 1 == b is in TMEM
+  uint64_t* p_full = bars + 9;    // [2] P^T of those items written back (bf16)
+  uint64_t* dp_full = bars + 11;  // dP^T of the current item is in TMEM
+  uint64_t* ds_full = bars + 12;  // dS^T of the current item written back (bf16)
+  uint64_t* ld_full = bars + 13;  // [2]
+  uint64_t* done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
   float* sLD = reinterpret_cast<float*>(smem + kBtOffLD);
 
   // key tiles in ascending order, KV heads fastest: the longest causal loops start first
@@ -92,9 +120,13 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         mbar_init(&q_full[i], 1);
         mbar_init(&q_empty[i], 1);
       }
-      for (int i = 0; i < 2; ++i) mbar_init(&ld_full[i], 128);
-      mbar_init(s_full, 1);
-      mbar_init(p_full, 128);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&ld_full[i], 128);
+        mbar_init(&s_full[i], 1);
+        mbar_init(&p_full[i], 128);
+      }
+      mbar_init(dp_full, 1);
+      mbar_init(ds_full, 128);
       mbar_init(done, 1);
       *abort_flag = timed_out_before() ? 1 : 0;
       fence_mbar_init();
@@ -171,23 +203,30 @@ __global__ void __launch_bounds__(kBtThreads, 1)
           umma_ss_lo(tDP, dV + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
                      b + ((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), dhi, id_s, kk > 0 ? 1u : 0u);
       };
-      // dV += P^T dO, dK += dS^T Q: 4 K-steps of 16 queries (A: 8 TMEM columns; B: 16 rows = 2 KB)
-      auto issue_acc = [&](int j, int st) {
-        const uint32_t tP = tS(j);
-        const uint32_t bo = dOm0 + st * kStageStep, bq = dQm0 + st * kStageStep;
+      // dV += P^T dO and dK += dS^T Q: 4 K-steps of 16 queries each (A: 8 TMEM
+      // columns; B: 16 rows = 2 KB)
+      auto issue_dv = [&](int j, int st) {
+        const uint32_t tP = tS(j), bo = dOm0 + st * kStageStep;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ts_lo(tDV, tP + kk * 8, bo + ((kk * 2048) >> 4), dhi, id_v, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dk = [&](int j, int st) {
+        const uint32_t bq = dQm0 + st * kStageStep;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_ts_lo(tDK, tDP + kk * 8, bq + ((kk * 2048) >> 4), dhi, id_k, (j > 0 || kk > 0) ? 1u : 0u);
       };
+      // Per item j the softmax hands over P^T first (-> dV) and dS^T second
+      // (-> dK); the next item's S^T is issued one item ahead into the other
+      // buffer, its dP^T once dK has consumed the dP buffer.
       bool ok = wait_bounded(kv_full, 0, abort_flag) && wait_bounded(&q_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(tS(0), 0);
+        umma_commit(&s_full[0]);
         issue_dp(0);
-        umma_commit(s_full);
+        umma_commit(dp_full);
       }
       for (int j = 0; ok && j < items; ++j) {
         const int st = j % kBtStages;
@@ -197,14 +236,18 @@ __global__ void __launch_bounds__(kBtThreads, 1)
           if (!(ok = wait_bounded(&q_full[sn], ((j + 1) / kBtStages) & 1, abort_flag))) break;
           tc_fence_after();
           issue_s(tS(j + 1), sn);  // overlaps the softmax of item j
+          umma_commit(&s_full[(j + 1) & 1]);
         }
-        if (!(ok = wait_bounded(p_full, j & 1, abort_flag))) break;
+        if (!(ok = wait_bounded(&p_full[j & 1], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc(j, st);
+        issue_dv(j, st);
+        if (!(ok = wait_bounded(ds_full, j & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_dk(j, st);
         umma_commit(&q_empty[st]);
         if (more) {
           issue_dp(sn);
-          umma_commit(s_full);
+          umma_commit(dp_full);
         }
       }
       if (ok) umma_commit(done);
@@ -231,37 +274,54 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       mbar_arrive(&ld_full[j & 1]);
       if (j + 1 < items) nxt = fetch(j + 1);  // in flight during this item
       if (!(ok = wait_bounded(&ld_full[j & 1], (j >> 1) & 1, abort_flag))) break;
-      if (!(ok = wait_bounded(s_full, j & 1, abort_flag))) break;
+      // visible query columns of this key row: [c_lo, c_hi] (empty when c_hi < c_lo)
+      const int c_lo = max(key - q0, 0);
+      int c_hi = min(len - 1 - q0, kBtQ - 1);
+      if (p.window > 0) c_hi = min(c_hi, key + p.window - 1 - q0);
+      if (key >= len) c_hi = -1;
+      // one branch per warp and item: every row sees every query, or selects per element
+      const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == kBtQ - 1);
+      // ---- P^T = 2^(S^T s log2e - lse log2e), rounded to bf16 over S^T -> dV
+      if (!(ok = wait_bounded(&s_full[j & 1], (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
       const uint32_t tSr = tbase + lane_off + ((j & 1) ? kBtColS1 : kBtColS0);
       const uint32_t tDPr = tbase + lane_off + kBtColDP;
-      float s[64], dp[64];
-      tmem_load64_sync(tSr, s);
-      tmem_load64_sync(tDPr, dp);
-      // every query of the item sees this key: no per-element mask
-      const bool full = key < len && q0 >= key && q0 + kBtQ - 1 < len &&
-                        (p.window == 0 || q0 + kBtQ - 1 - key <= p.window - 1);
-      uint32_t pk[32], dk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float pe[2], de[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int qc = 2 * c + e;
-          const int qp = q0 + qc;
-          const bool vis = full || (key < len && qp < len && bw_visible(qp, key, p.window));
-          const float pr = vis ? ex2(fmaf(s[qc], p.scale_log2, -ld[qc])) : 0.f;
-          pe[e] = pr;
-          de[e] = vis ? pr * (p.v_scale * dp[qc] - ld[kBtQ + qc]) : 0.f;
-        }
-        pk[c] = pack_bf16(pe[0], pe[1]);
-        dk[c] = pack_bf16(de[0], de[1]);
+      const float4* ld4 = reinterpret_cast<const float4*>(ld);  // [0,16): lse log2e, [16,32): D
+      float pe[64];
+      tmem_load64_sync(tSr, pe);
+      {
+        uint32_t pk[32];
+        if (full)
+          bwd_p_tile<false>(pe, ld4, p.scale_log2, c_lo, c_hi, pk);
+        else
+          bwd_p_tile<true>(pe, ld4, p.scale_log2, c_lo, c_hi, pk);
+        tmem_st32(tSr, pk);
       }
-      tmem_st32(tSr, pk);
-      tmem_st32(tDPr, dk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
+      // ---- dS^T = P^T (v_scale dP^T - D), rounded to bf16 over dP^T -> dK
+      if (!(ok = wait_bounded(dp_full, j & 1, abort_flag))) break;
+      tc_fence_after();
+      {
+        float dp[64];
+        tmem_load64_sync(tDPr, dp);
+        uint32_t dk[32];
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 d4 = ld4[16 + c4];
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float de[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) de[e] = pe[4 * c4 + e] * fmaf(p.v_scale, dp[4 * c4 + e], -dv4[e]);
+          dk[2 * c4] = pack_bf16(de[0], de[1]);
+          dk[2 * c4 + 1] = pack_bf16(de[2], de[3]);
+        }
+        tmem_st32(tDPr, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full);
     }
     // ---------------- epilogue: dV * v_scale and dK * scale for valid keys
     if (ok && wait_bounded(done, 0, abort_flag)) {

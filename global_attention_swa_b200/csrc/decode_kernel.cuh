@@ -25,12 +25,17 @@
 namespace mimo {
 
 constexpr int kDecTileKeys = 64;
-constexpr int kDecStages = 4;
+constexpr int kDecStages = 4;                        // long caches: one CTA per SM
+constexpr int kDecShortStages = 2;                   // short caches (rings): two CTAs per SM
+constexpr int kDecShortKeys = 256;                   // "short": at most this many visible slots
 constexpr int kDecKBytes = kDecTileKeys * 192 * 2;   // 24576
 constexpr int kDecVBytes = kDecTileKeys * 128 * 2;   // 16384
 constexpr int kDecStageBytes = kDecKBytes + kDecVBytes;
 constexpr int kDecThreads = 160;                     // 4 consumer warps + 1 producer warp
-constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 /*align*/ + 128 /*barriers*/;
+constexpr int dec_smem_bytes(int stages) { return stages * kDecStageBytes + 1024 /*align*/ + 128 /*barriers*/; }
+constexpr int kDecSmemBytes = dec_smem_bytes(kDecStages);
+// the end-of-split merge reuses the stage ring: [4 warps][16 rows][128] + 3 x [4][16] floats
+static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kDecShortStages * kDecStageBytes, "merge buffer fits");
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // [B, Hq, 192]
@@ -71,15 +76,20 @@ __device__ __forceinline__ void decode_range(const DecodeParams& p, int L, int& 
   }
 }
 
-__global__ void __launch_bounds__(kDecThreads, 1)
+// kStages shared-memory stages of one 64-key K/V tile each; kCtasPerSm CTAs
+// resident per SM.  Long caches stream through 4 stages at one CTA per SM; a
+// short cache (a 129-slot ring: three tiles) has little to pipeline, and two
+// CTAs per SM with 2 stages each let all of a batch's units run in one wave.
+template <int kStages, int kCtasPerSm>
+__global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kDecStages * kDecStageBytes);
-  uint64_t* empty = full + kDecStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kDecStageBytes);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,7 +102,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int nkeys = max(0, s1 - s0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 4);
     }
@@ -112,9 +122,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tma_prefetch_desc(&tm_v);
       const int row0 = b * p.C + s0;
       for (int t = 0; t < ntiles; ++t) {
-        const int st = t % kDecStages;
-        if (t >= kDecStages) {
-          if (!wait_bounded(&empty[st], ((t / kDecStages) - 1) & 1, abort_flag)) break;
+        const int st = t % kStages;
+        if (t >= kStages) {
+          if (!wait_bounded(&empty[st], ((t / kStages) - 1) & 1, abort_flag)) break;
         }
         uint8_t* kb = smem + st * kDecStageBytes;
         uint8_t* vb = kb + kDecKBytes;
@@ -156,8 +166,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int kw = warp * 16;  // this warp's 16 keys within each tile
     const uint32_t sbase = smem_u32(smem);
     for (int t = 0; t < ntiles; ++t) {
-      const int st = t % kDecStages;
-      if (!wait_bounded(&full[st], (t / kDecStages) & 1, abort_flag)) break;
+      const int st = t % kStages;
+      if (!wait_bounded(&full[st], (t / kStages) & 1, abort_flag)) break;
       const int valid = min(kDecTileKeys, nkeys - t * kDecTileKeys);
       if (kw < valid) {
         const uint32_t kb = sbase + st * kDecStageBytes;

@@ -162,7 +162,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
                       it.g * p.G, it.b0 + it.q0 + blk * p.QB);
       };
       // Blocks are numbered n = 0, 1, ... over this CTA's pairs; block n uses Q
-      // buffer n & 1.  The pair's K/V window is loaded at its first block.
+      // buffer n & 1.  The pair's K/V window is loaded at its first block.  The
+      // next pair's Q and K/V are prefetched into L2 when a pair starts, two
+      // blocks ahead of their loads (a Q tile from DRAM takes longer than one
+      // block's work, and there is no room for a third Q buffer).
       SwItem cur, nxt;
       int r = sw_next(p, 0, rounds, cur);
       if (r >= 0) load_q(cur, 0, 0);
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       int n = 0, kp = 0;
       while (ok && r >= 0) {
         const int k0 = cur.q0 + 2 * p.QB - N;  // may be negative: zero-filled or masked
-        int rn = -1;
+        const int rn = sw_next(p, r + 1, rounds, nxt);
         for (int blk = 0; ok && blk < cur.nblk; ++blk, ++n) {
           if (blk == 0) {
             if (kp >= 1 && !(ok = wait_bounded(k_empty, (kp - 1) & 1, abort_flag))) break;
@@ -178,11 +181,21 @@ __global__ void __launch_bounds__(kSwThreads, 1)
 #pragma unroll
             for (int c = 0; c < 3; ++c)
               tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
+            if (rn >= 0) {
+              const int nk0 = nxt.b0 + nxt.q0 + 2 * p.QB - N;
+#pragma unroll
+              for (int c = 0; c < 3; ++c) {
+                for (int b = 0; b < nxt.nblk; ++b)
+                  tma_prefetch_l2_3d(&tm_q, c * 64, nxt.g * p.G, nxt.b0 + nxt.q0 + b * p.QB);
+                tma_prefetch_l2_3d(&tm_k, c * 64, nxt.g, nk0);
+              }
+#pragma unroll
+              for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_v, c * 64, nxt.g, nk0);
+            }
           }
           // the next block's Q, one block ahead (its buffer was freed by S(n-1))
           const int bn = (n + 1) & 1;
           const bool next_in_pair = (blk + 1 < cur.nblk);
-          if (!next_in_pair) rn = sw_next(p, r + 1, rounds, nxt);
           if (next_in_pair || rn >= 0) {
             if (n + 1 >= 2 && !(ok = wait_bounded(&q_empty[bn], (((n + 1) >> 1) - 1) & 1, abort_flag))) break;
             if (next_in_pair)

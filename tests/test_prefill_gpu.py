@@ -60,6 +60,33 @@ def test_varlen_pack_with_empty_and_single_token_sequences(window):
     P.check(out, ro, lse, rl, what=f"varlen W={window}")
 
 
+# query heads in groups of four per key/value head run on CTA pairs (M = 256
+# MMAs, two heads per CTA); groups of 8 with a window the packed kernel cannot
+# hold (N > 192), and groups of 4 with any window, take the pair kernel too
+
+
+@pytest.mark.parametrize("hq,hkv,window", [(8, 2, 0), (8, 2, 1), (8, 2, 2), (8, 2, 129),
+                                           (32, 2, 0), (32, 4, 300), (4, 1, 128)])
+def test_pair_kernel_lengths(hq, hkv, window):
+    for T in (1, 2, 127, 128, 129, 255, 256, 257, 1000):
+        sinks = (T + window) % 2 == 1
+        x = W.prefill_inputs([T], hq=hq, hkv=hkv, seed=T * 13 + window + hq, sinks=sinks)
+        out_dtype = torch.bfloat16 if T % 3 == 0 else torch.float32
+        out, lse = run_gpu(x, window, out_dtype)
+        ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+        P.check(out, ro, lse, rl, what=f"pair Hq={hq} Hkv={hkv} T={T} W={window}")
+
+
+def test_pair_kernel_many_items_per_cluster_varlen():
+    """More items than CTA pairs, with sequences of every length class packed."""
+    lengths = [1, 1000, 0, 129, 2000, 127, 3, 700, 128, 1500]
+    x = W.prefill_inputs(lengths, hq=16, hkv=2, seed=61)
+    for window in (0, 500):
+        out, lse = run_gpu(x, window, torch.float32)
+        ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+        P.check(out, ro, lse, rl, what=f"pair varlen W={window}")
+
+
 def test_varlen_pack_equals_separate_calls():
     lengths = [200, 1, 513]
     x = W.prefill_inputs(lengths, hq=8, hkv=2, seed=5)
