@@ -150,13 +150,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
       }
       fence_mbar_init();
     }
-    __syncwarp();
+  }
+  cluster_sync();  // both CTAs running, their barriers initialised
+  if (warp == 8) {
+    // the same warp of both CTAs allocates for the pair (the address lands in both)
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
-  tc_fence_before();
-  cluster_sync();  // both CTAs running, their barriers initialised, TMEM allocated
-  tc_fence_after();
   if (threadIdx.x == 0) {
     // both CTAs take the same decision: each publishes its own reading of the
     // device status word to both CTAs, and both act on the union
@@ -164,7 +164,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
     for (uint32_t r = 0; r < 2; ++r)
       st_shared_cluster_u32(mapa_shared(smem_u32((const void*)&abort_seen[rank]), r), seen);
   }
-  cluster_sync();
+  tc_fence_before();
+  cluster_sync();  // TMEM allocated, abort readings exchanged
+  tc_fence_after();
   if (threadIdx.x == 0) *abort_flag = (abort_seen[0] | abort_seen[1]) ? 1 : 0;
   __syncthreads();
   const uint32_t tbase = *tmem_slot;
