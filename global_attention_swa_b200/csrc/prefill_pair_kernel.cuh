@@ -293,7 +293,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           if (!(ok = wait_bounded(&k_full[g_t & 1], (g_t >> 1) & 1, abort_flag))) break;
 #pragma unroll 1
           for (int i = 0; i < 2; ++i) {
-            if (g_t > 0 && !(ok = wait_bounded(&s_free[i], (g_t - 1) & 1, abort_flag))) break;
+            if (g_t > 0 && !(ok = wait_bounded_cluster(&s_free[i], (g_t - 1) & 1, abort_flag))) break;
             tc_fence_after();
             issue_s(i, g_t & 1);
             umma_commit_pair(&s_full[i], kBoth);
@@ -307,8 +307,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
             if (!(ok = wait_bounded(v_full, g_p & 1, abort_flag))) break;
 #pragma unroll 1
             for (int i = 0; i < 2; ++i) {
-              if (!(ok = wait_bounded(&p_full[i], g_p & 1, abort_flag))) break;
-              if (t == 1 && n > 0 && !(ok = wait_bounded(&o_empty[i], (n - 1) & 1, abort_flag))) break;
+              if (!(ok = wait_bounded_cluster(&p_full[i], g_p & 1, abort_flag))) break;
+              if (t == 1 && n > 0 && !(ok = wait_bounded_cluster(&o_empty[i], (n - 1) & 1, abort_flag))) break;
               tc_fence_after();
               issue_pv(i, t > 1);
               umma_commit_pair(&pv_done[i], kBoth);
@@ -324,8 +324,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           if (!(ok = wait_bounded(v_full, g_p & 1, abort_flag))) break;
 #pragma unroll 1
           for (int i = 0; i < 2; ++i) {
-            if (!(ok = wait_bounded(&p_full[i], g_p & 1, abort_flag))) break;
-            if (it.n_kt == 1 && n > 0 && !(ok = wait_bounded(&o_empty[i], (n - 1) & 1, abort_flag))) break;
+            if (!(ok = wait_bounded_cluster(&p_full[i], g_p & 1, abort_flag))) break;
+            if (it.n_kt == 1 && n > 0 && !(ok = wait_bounded_cluster(&o_empty[i], (n - 1) & 1, abort_flag))) break;
             tc_fence_after();
             issue_pv(i, it.n_kt > 1);
             umma_commit_pair(&pv_done[i], kBoth);
