@@ -34,8 +34,9 @@
 //
 // Barriers: loads are counted on the leader's full barriers (the leader's
 // producer expects the bytes of both CTAs); MMA completions arrive on both
-// CTAs' barriers (commit with a CTA mask); softmax and epilogue threads of
-// both CTAs arrive on the leader's barriers.  The softmax is the one of the
+// CTAs' barriers (commit with a CTA mask); each softmax / epilogue warp of both
+// CTAs arrives once (one lane, after every lane fenced its own accesses and
+// the warp synchronised) on the leader's barriers.  The softmax is the one of the
 // single-CTA kernel (prefill_kernel.cuh): base 2, the sink folded into the
 // running max and sum, conditional rescaling of O, the output normalised by
 // the sum of the bf16-rounded P.  Every wait is bounded.
@@ -142,9 +143,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
       for (int i = 0; i < 2; ++i) {
         mbar_init(&k_full[i], 1);
         mbar_init(&k_empty[i], 1);
-        mbar_init(&s_free[i], 256);
-        mbar_init(&p_full[i], 256);
-        mbar_init(&o_empty[i], 256);
+        mbar_init(&s_free[i], 8);   // one elected lane per softmax warp of both CTAs
+        mbar_init(&p_full[i], 8);   // one elected lane per softmax warp of both CTAs
+        mbar_init(&o_empty[i], 8);   // one elected lane per softmax warp of both CTAs
         mbar_init(&s_full[i], 1);
         mbar_init(&pv_done[i], 1);
       }
@@ -369,7 +370,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
         float s[128];
         tmem_load128_sync(tS, s);
         tc_fence_before();
-        mbar_arrive_cluster(b_sfree);  // S_i may now be overwritten by the next tile's scores
+        __syncwarp();
+        // S_i may now be overwritten by the next tile's scores (the loads are complete)
+        if (lane == 0) mbar_arrive_cluster_relaxed(b_sfree);
         const bool full_tile = (kpos0 + kPfTile - 1 <= it.q0) &&
                                (p.window == 0 || (it.q0 + kPfTile - 1) - kpos0 <= p.window - 1);
         float mx8[8];
@@ -440,7 +443,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive_cluster(b_pfull);
+        __syncwarp();
+        // the leader's own P tile needs only CTA-scope ordering; the peer's, cluster scope
+        if (lane == 0) {
+          if (rank == 0)
+            mbar_arrive(&p_full[i]);
+          else
+            mbar_arrive_cluster(b_pfull);
+        }
       }
       if (!ok) break;
       // ---------------- epilogue: O / l -> out, lse (O read out of TMEM and released first)
@@ -451,7 +461,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
       float o[128];
       tmem_load128_sync(tO, o);
       tc_fence_before();
-      mbar_arrive_cluster(b_oempty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(b_oempty);  // O read (loads complete)
       ++n;
       if (qpos < it.len) {
         const int tok = it.b0 + qpos;
