@@ -32,7 +32,12 @@ constexpr int kDecKBytes = kDecTileKeys * 192 * 2;   // 24576
 constexpr int kDecVBytes = kDecTileKeys * 128 * 2;   // 16384
 constexpr int kDecStageBytes = kDecKBytes + kDecVBytes;
 constexpr int kDecThreads = 160;                     // 4 consumer warps + 1 producer warp
-constexpr int dec_smem_bytes(int stages) { return stages * kDecStageBytes + 1024 /*align*/ + 128 /*barriers*/; }
+constexpr int dec_smem_bytes(int stages, int tile_rows = kDecTileKeys) {
+  return stages * 5 * tile_rows * 128 + 1024 /*align*/ + 128 /*barriers*/;
+}
+constexpr int kDecRingStages = 3;                    // small rings: the whole ring in flight
+constexpr int kDecRingRows = 48;                     // rows of a ring tile (3 x 48 >= 129 slots)
+static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kDecRingStages * 5 * kDecRingRows * 128, "merge buffer fits");
 constexpr int kDecSmemBytes = dec_smem_bytes(kDecStages);
 // the end-of-split merge reuses the stage ring: [4 warps][16 rows][128] + 3 x [4][16] floats
 static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kDecShortStages * kDecStageBytes, "merge buffer fits");
@@ -50,6 +55,8 @@ struct DecodeParams {
   int ring;     // 1: ring cache (C == window)
   int chunk;    // keys per split, multiple of 64
   int nsplit;   // splits per (b, g)
+  int tile;     // keys per tile (rows of the K / V TMA boxes): 64, or at most 48 for a small ring
+  int spec_tiles;  // > 0: stream this many tiles from slot 0 without waiting for the length (small rings)
   float scale_log2;  // softmax_scale * log2(e)
   float v_scale;
   int out_f32;
@@ -76,18 +83,24 @@ __device__ __forceinline__ void decode_range(const DecodeParams& p, int L, int& 
   }
 }
 
-// kStages shared-memory stages of one 64-key K/V tile each; kCtasPerSm CTAs
-// resident per SM.  Long caches stream through 4 stages at one CTA per SM; a
-// short cache (a 129-slot ring: three tiles) has little to pipeline, and two
-// CTAs per SM with 2 stages each let all of a batch's units run in one wave.
-template <int kStages, int kCtasPerSm>
+// kStages shared-memory stages of one K/V tile of at most kTileRows keys each
+// (p.tile keys, the rows of the TMA boxes); kCtasPerSm CTAs resident per SM.
+// Long caches stream 64-key tiles through 4 stages at one CTA per SM.  Short
+// caches have little to pipeline: two CTAs per SM let all of a batch's units
+// run in one wave, and a small ring (at most 3 x 48 slots, e.g. 129) is
+// loaded whole, in three tiles issued at once without waiting for the
+// sequence length (a ring's visible slots always start at slot 0; the length
+// only masks keys).
+template <int kStages, int kCtasPerSm, int kTileRows>
 __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   extern __shared__ __align__(1024) uint8_t dsmem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kDecStageBytes);
+  constexpr int kBox = kTileRows * 128;          // one [rows][64 dims] swizzled box
+  constexpr int kStageBytes = 5 * kBox;          // K: 3 boxes, V: 2 boxes
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
 
@@ -113,7 +126,9 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   __syncthreads();
   // after a recorded timeout elsewhere, return at entry: nothing is read or written
   if (*abort_flag) return;
-  const int ntiles = (nkeys + kDecTileKeys - 1) / kDecTileKeys;
+  const int tile = p.tile;
+  // tiles streamed: those holding the unit's keys, or every tile of a small ring
+  const int ntiles = p.spec_tiles > 0 ? p.spec_tiles : (nkeys + tile - 1) / tile;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -126,14 +141,14 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
         if (t >= kStages) {
           if (!wait_bounded(&empty[st], ((t / kStages) - 1) & 1, abort_flag)) break;
         }
-        uint8_t* kb = smem + st * kDecStageBytes;
-        uint8_t* vb = kb + kDecKBytes;
-        mbar_arrive_expect_tx(&full[st], kDecStageBytes);
-        const int y = row0 + t * kDecTileKeys;
+        uint8_t* kb = smem + st * kStageBytes;
+        uint8_t* vb = kb + 3 * kBox;
+        mbar_arrive_expect_tx(&full[st], 5 * tile * 128);
+        const int y = row0 + t * tile;
 #pragma unroll
-        for (int c = 0; c < 3; ++c) tma_load_2d(kb + c * 8192, &tm_k, &full[st], g * 192 + c * 64, y);
+        for (int c = 0; c < 3; ++c) tma_load_2d(kb + c * kBox, &tm_k, &full[st], g * 192 + c * 64, y);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) tma_load_2d(vb + c * 8192, &tm_v, &full[st], g * 128 + c * 64, y);
+        for (int c = 0; c < 2; ++c) tma_load_2d(vb + c * kBox, &tm_v, &full[st], g * 128 + c * 64, y);
       }
     }
   } else {
@@ -168,10 +183,10 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     for (int t = 0; t < ntiles; ++t) {
       const int st = t % kStages;
       if (!wait_bounded(&full[st], (t / kStages) & 1, abort_flag)) break;
-      const int valid = min(kDecTileKeys, nkeys - t * kDecTileKeys);
+      const int valid = min(tile, nkeys - t * tile);  // may be <= 0 for a ring's spare tile
       if (kw < valid) {
-        const uint32_t kb = sbase + st * kDecStageBytes;
-        const uint32_t vb = kb + kDecKBytes;
+        const uint32_t kb = sbase + st * kStageBytes;
+        const uint32_t vb = kb + 3 * kBox;
         // ---- S = Q K^T for keys kw .. kw+15 (two n-blocks of 8)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {
@@ -184,7 +199,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
             const int c = kk >> 2;                       // 64-dim box
             const int col = (kk & 3) * 16 + kcol;
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(kb + c * 8192 + sw128_offset(krow, col), b0, b1, b2, b3);
+            ldsm_x4(kb + c * kBox + sw128_offset(krow, col), b0, b1, b2, b3);
             mma_bf16_16816(s[0], qa[kk], b0, b1);
             mma_bf16_16816(s[1], qa[kk], b2, b3);
           }
@@ -250,7 +265,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
           const int c = n2 >> 2;  // 64-dim box
           const int col = (n2 & 3) * 16 + vcol;
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vb + c * 8192 + sw128_offset(vrow, col), b0, b1, b2, b3);
+          ldsm_x4_t(vb + c * kBox + sw128_offset(vrow, col), b0, b1, b2, b3);
           if (partial) {  // invalid slots may hold anything: zero them
             b0 &= mk0; b1 &= mk1; b2 &= mk0; b3 &= mk1;
           }

@@ -146,15 +146,20 @@ mimo_status_t ensure_attributes() {
                                             mimo::kSwSmemBytes),
                        "sliding-window prefill smem attribute")))
     return st;
-  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel<mimo::kDecStages, 1>,
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel<mimo::kDecStages, 1, mimo::kDecTileKeys>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kDecSmemBytes),
                        "decode smem attribute")))
     return st;
-  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel<mimo::kDecShortStages, 2>,
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel<mimo::kDecShortStages, 2, mimo::kDecTileKeys>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::dec_smem_bytes(mimo::kDecShortStages)),
                        "short-cache decode smem attribute")))
+    return st;
+  if ((st = cuda_check(cudaFuncSetAttribute(mimo::decode_split_kernel<mimo::kDecRingStages, 2, mimo::kDecRingRows>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            mimo::dec_smem_bytes(mimo::kDecRingStages, mimo::kDecRingRows)),
+                       "ring decode smem attribute")))
     return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::bwd_dq_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -486,13 +491,23 @@ mimo_status_t decode_impl(const mimo_attn_dims_t* dims, const void* q, const voi
     return fail(MIMO_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if ((st = ensure_attributes())) return st;
 
+  // A small ring (at most 3 x 48 slots, e.g. the 129-slot sliding-window cache)
+  // is streamed whole in three equal tiles (43 rows for 129 slots), issued
+  // before the sequence length is known.
+  const bool small_ring = !fp8 && pl.ring && pl.nsplit == 1 &&
+                          capacity <= mimo::kDecRingStages * mimo::kDecRingRows;
+  int tile = mimo::kDecTileKeys, spec_tiles = 0;
+  if (small_ring) {
+    spec_tiles = (capacity + mimo::kDecRingRows - 1) / mimo::kDecRingRows;
+    tile = (capacity + spec_tiles - 1) / spec_tiles;
+  }
   CUtensorMap tk, tv;
   {
     // bf16: boxes of 64 elements (128 B, 128-byte swizzle); e4m3: 64 bytes, 64-byte swizzle
     const int eb = fp8 ? 1 : 2;
     const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle sw = fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-    const uint32_t rows = fp8 ? (uint32_t)mimo::kD8TileKeys : (uint32_t)mimo::kDecTileKeys;
+    const uint32_t rows = fp8 ? (uint32_t)mimo::kD8TileKeys : (uint32_t)tile;
     {
       const uint64_t d[2] = {(uint64_t)Hkv * 192, (uint64_t)batch * capacity};
       const uint64_t s[1] = {(uint64_t)Hkv * 192 * eb};
@@ -524,6 +539,8 @@ mimo_status_t decode_impl(const mimo_attn_dims_t* dims, const void* q, const voi
   p.ring = pl.ring;
   p.chunk = pl.chunk;
   p.nsplit = pl.nsplit;
+  p.tile = tile;
+  p.spec_tiles = spec_tiles;
   p.scale_log2 = scale_log2_of(dims);
   p.v_scale = v_scale_of(dims);
   p.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
@@ -533,11 +550,15 @@ mimo_status_t decode_impl(const mimo_attn_dims_t* dims, const void* q, const voi
   if (fp8)
     mimo::decode_split_fp8_kernel<<<grid, mimo::kD8Threads, mimo::kD8SmemBytes, (cudaStream_t)stream>>>(
         tk, tv, p);
+  else if (small_ring)
+    mimo::decode_split_kernel<mimo::kDecRingStages, 2, mimo::kDecRingRows>
+        <<<grid, mimo::kDecThreads, mimo::dec_smem_bytes(mimo::kDecRingStages, mimo::kDecRingRows),
+           (cudaStream_t)stream>>>(tk, tv, p);
   else if (pl.cap_eff <= mimo::kDecShortKeys)
-    mimo::decode_split_kernel<mimo::kDecShortStages, 2>
+    mimo::decode_split_kernel<mimo::kDecShortStages, 2, mimo::kDecTileKeys>
         <<<grid, mimo::kDecThreads, mimo::dec_smem_bytes(mimo::kDecShortStages), (cudaStream_t)stream>>>(tk, tv, p);
   else
-    mimo::decode_split_kernel<mimo::kDecStages, 1>
+    mimo::decode_split_kernel<mimo::kDecStages, 1, mimo::kDecTileKeys>
         <<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, (cudaStream_t)stream>>>(tk, tv, p);
   if ((st = cuda_check(cudaGetLastError(), "decode launch"))) return st;
   if (pl.nsplit > 1) {

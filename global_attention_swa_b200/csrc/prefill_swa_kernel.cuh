@@ -294,58 +294,70 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       if (!(ok = wait_bounded(&s_full[b], (n >> 1) & 1, abort_flag))) break;
       tc_fence_after();
       const uint32_t tS = tbase + lane_off + b * kSwNMax;
-      // pass 1: row max over the visible columns
+      // pass 1: row max over the visible columns.  The row is read in chunks of
+      // 48 columns (one wait per chunk); columns at or past N lie outside
+      // [c_lo, c_hi] and are masked like the window's edges.
       float mx0 = -INFINITY, mx1 = -INFINITY;
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t v[16];
-        tmem_load16_sync(tS + c0, v);
-        if (c0 >= c_lo && c0 + 15 <= c_hi) {
+      for (int c0 = 0; c0 < N; c0 += 48) {
+        uint32_t v[48];
+        tmem_load48_sync(tS + c0, v);
 #pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            mx0 = fmax3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-            mx1 = fmax3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-          }
-        } else {
+        for (int q = 0; q < 3; ++q) {
+          const int cq0 = c0 + 16 * q;
+          if (cq0 >= c_lo && cq0 + 15 <= c_hi) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = c0 + e;
-            if (c >= c_lo && c <= c_hi) mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+            for (int e = 0; e < 16; e += 4) {
+              mx0 = fmax3(mx0, __uint_as_float(v[16 * q + e]), __uint_as_float(v[16 * q + e + 1]));
+              mx1 = fmax3(mx1, __uint_as_float(v[16 * q + e + 2]), __uint_as_float(v[16 * q + e + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = cq0 + e;
+              if (c >= c_lo && c <= c_hi) mx0 = fmaxf(mx0, __uint_as_float(v[16 * q + e]));
+            }
           }
         }
       }
       const float m = fmaxf(sg2, fmaxf(mx0, mx1) * p.scale_log2);
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same
-      // columns.  The unrounded sum gives lse; the sum of the rounded P (the
-      // values P.V multiplies) normalises the output.
+      // columns (P of columns [c0, c0 + 48) lands in [c0 / 2, c0 / 2 + 24), behind
+      // the read position).  The unrounded sum gives lse; the sum of the rounded
+      // P (the values P.V multiplies) normalises the output.
       float2 l2 = make_float2(0.f, 0.f), lr2 = make_float2(0.f, 0.f);
-      for (int c0 = 0; c0 < N; c0 += 16) {
-        uint32_t v[16], pk[8];
-        tmem_load16_sync(tS + c0, v);
-        if (c0 >= c_lo && c0 + 15 <= c_hi) {
+      for (int c0 = 0; c0 < N; c0 += 48) {
+        uint32_t v[48];
+        tmem_load48_sync(tS + c0, v);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 x = fma2(make_float2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])),
-                                  make_float2(p.scale_log2, p.scale_log2), make_float2(neg_m, neg_m));
-            const float2 pe = make_float2(ex2(x.x), ex2(x.y));
-            pk[e] = pack_bf16(pe.x, pe.y);
-            l2 = add2(l2, pe);
-            lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
-          }
-        } else {
+        for (int q = 0; q < 3; ++q) {
+          const int cq0 = c0 + 16 * q;
+          uint32_t pk[8];
+          if (cq0 >= c_lo && cq0 + 15 <= c_hi) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = c0 + 2 * e;
-            const float x0 = fmaf(__uint_as_float(v[2 * e]), p.scale_log2, neg_m);
-            const float x1 = fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, neg_m);
-            const float2 pe = make_float2((c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f,
-                                          (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f);
-            pk[e] = pack_bf16(pe.x, pe.y);
-            l2 = add2(l2, pe);
-            lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
+            for (int e = 0; e < 8; ++e) {
+              const float2 x = fma2(make_float2(__uint_as_float(v[16 * q + 2 * e]), __uint_as_float(v[16 * q + 2 * e + 1])),
+                                    make_float2(p.scale_log2, p.scale_log2), make_float2(neg_m, neg_m));
+              const float2 pe = make_float2(ex2(x.x), ex2(x.y));
+              pk[e] = pack_bf16(pe.x, pe.y);
+              l2 = add2(l2, pe);
+              lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = cq0 + 2 * e;
+              const float x0 = fmaf(__uint_as_float(v[16 * q + 2 * e]), p.scale_log2, neg_m);
+              const float x1 = fmaf(__uint_as_float(v[16 * q + 2 * e + 1]), p.scale_log2, neg_m);
+              const float2 pe = make_float2((c >= c_lo && c <= c_hi) ? ex2(x0) : 0.f,
+                                            (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f);
+              pk[e] = pack_bf16(pe.x, pe.y);
+              l2 = add2(l2, pe);
+              lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
+            }
           }
+          if (cq0 < N) tmem_st8(tS + cq0 / 2, pk);
         }
-        tmem_st8(tS + c0 / 2, pk);
       }
       tmem_wait_st();
       tc_fence_before();
