@@ -18,9 +18,9 @@
 // softmax warps compute the exponentials of tile t+1.
 //
 //   warp 8      TMA producer of this CTA's Q_0, Q_1 and half K tiles
-//   warp 9      MMA issuer (one thread, leader CTA only)
+//   warp 9      score-MMA issuer (one thread, leader CTA only)
 //   warp 10     TMA producer of this CTA's half V tiles
-//   warp 11     idle (it completes the third warpgroup)
+//   warp 11     P.V-MMA issuer (one thread, leader CTA only)
 //   warps 0-3   softmax + epilogue of slot 0 (TMEM lanes 0..127, one row each)
 //   warps 4-7   softmax + epilogue of slot 1
 //
@@ -247,95 +247,93 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
         ++n;
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer (leader)
+  } else if (warp == 9 || warp == 11) {
+    // ------------------------------------------------------------ MMA issuers (leader)
+    // Two threads feed the tensor pipe: warp 9 issues the score products, warp
+    // 11 the P.V products.  The two streams never touch the same TMEM columns
+    // or shared memory (S_i vs O_i; Q, K vs P, V), so neither needs the other's
+    // order, and while one waits on a barrier the other keeps the pipe busy (an
+    // issuing thread advances only as fast as the pipe takes its MMAs).
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(256, 128, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(256, 128, false, true);
       constexpr uint32_t dhi = desc_hi_sw128(1024);
-      // per-slot operands are the slot-0 ones plus a slot stride (no arrays: a
-      // runtime-indexed array would live in local memory)
-      const uint32_t dQ0 = desc_lo_sw128(sbase + kPpOffQ, 16);
-      const uint32_t dP0 = desc_lo_sw128(sbase + kPpOffP, 16);
-      const uint32_t dK0 = desc_lo_sw128(sbase + kPpOffK, 16);
-      const uint32_t dV = desc_lo_sw128(sbase + kPpOffV, 16384);  // MN-major, one 64-column atom per CTA
-      // S_i = Q_i K^T: 12 K-steps of 16 dims (A boxes 16 KB apart, B boxes 8 KB apart)
-      auto issue_s = [&](int i, int ks) {
-        const uint32_t a = dQ0 + static_cast<uint32_t>(i) * (kPpQBytes >> 4);
-        const uint32_t b = dK0 + static_cast<uint32_t>(ks) * (kPpKBytes >> 4);
-        const uint32_t d = tbase + static_cast<uint32_t>(i) * 128;
+      if (warp == 9) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(256, 128, false, false);
+        const uint32_t dQ0 = desc_lo_sw128(sbase + kPpOffQ, 16);
+        const uint32_t dK0 = desc_lo_sw128(sbase + kPpOffK, 16);
+        // S_i = Q_i K^T: 12 K-steps of 16 dims (A boxes 16 KB apart, B boxes 8 KB apart)
+        auto issue_s = [&](int i, int ks) {
+          const uint32_t a = dQ0 + static_cast<uint32_t>(i) * (kPpQBytes >> 4);
+          const uint32_t b = dK0 + static_cast<uint32_t>(ks) * (kPpKBytes >> 4);
+          const uint32_t d = tbase + static_cast<uint32_t>(i) * 128;
 #pragma unroll
-        for (int kk = 0; kk < 12; ++kk)
-          umma_ss_lo_pair(d, a + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                          b + ((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), dhi, idesc_s, kk > 0 ? 1u : 0u);
-      };
-      // O_i += P_i V: 8 K-steps of 16 keys (A boxes 16 KB apart; B: 16 key rows = 2 KB)
-      auto issue_pv = [&](int i, bool acc) {
-        const uint32_t a = dP0 + static_cast<uint32_t>(i) * (kPpPBytes >> 4);
-        const uint32_t d = tbase + 256 + static_cast<uint32_t>(i) * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss_lo_pair(d, a + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                          dV + ((kk * 2048) >> 4), dhi, idesc_o, (acc || kk > 0) ? 1u : 0u);
-      };
-      int n = 0;       // items
-      int kt = 0;      // key tiles over all items (K stages, V, slot tiles)
-      bool ok = true;
-      for (int r = 0; ok && r < rounds; ++r) {
-        const int item = pf_item_index(r, cl, nclusters);
-        if (item >= p.num_items) continue;
-        const PpItem it = pp_decode(p, item);
-        if (!it.valid) continue;
-        if (!(ok = wait_bounded(q_full, n & 1, abort_flag))) break;
-        for (int t = 0; ok && t < it.n_kt; ++t) {
-          const int g_t = kt + t;  // global tile index of tile t
-          // scores of tile t for both slots (slot buffers free once the
-          // softmax read the previous tile's scores)
-          if (!(ok = wait_bounded(&k_full[g_t & 1], (g_t >> 1) & 1, abort_flag))) break;
-#pragma unroll 1
-          for (int i = 0; i < 2; ++i) {
-            if (g_t > 0 && !(ok = wait_bounded_cluster(&s_free[i], (g_t - 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_s(i, g_t & 1);
-            umma_commit_pair(&s_full[i], kBoth);
-          }
-          if (!ok) break;
-          umma_commit_pair(&k_empty[g_t & 1], kBoth);
-          if (t == it.n_kt - 1) umma_commit_pair(q_empty, kBoth);
-          // P.V of the previous tile of this item
-          if (t > 0) {
-            const int g_p = g_t - 1;
-            if (!(ok = wait_bounded(v_full, g_p & 1, abort_flag))) break;
+          for (int kk = 0; kk < 12; ++kk)
+            umma_ss_lo_pair(d, a + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                            b + ((((kk >> 2) * 8192) + (kk & 3) * 32) >> 4), dhi, idesc_s, kk > 0 ? 1u : 0u);
+        };
+        int n = 0, kt = 0;
+        bool ok = true;
+        for (int r = 0; ok && r < rounds; ++r) {
+          const int item = pf_item_index(r, cl, nclusters);
+          if (item >= p.num_items) continue;
+          const PpItem it = pp_decode(p, item);
+          if (!it.valid) continue;
+          if (!(ok = wait_bounded(q_full, n & 1, abort_flag))) break;
+          for (int t = 0; ok && t < it.n_kt; ++t) {
+            const int g_t = kt + t;  // tile index over all items
+            if (!(ok = wait_bounded(&k_full[g_t & 1], (g_t >> 1) & 1, abort_flag))) break;
 #pragma unroll 1
             for (int i = 0; i < 2; ++i) {
-              if (!(ok = wait_bounded_cluster(&p_full[i], g_p & 1, abort_flag))) break;
-              if (t == 1 && n > 0 && !(ok = wait_bounded_cluster(&o_empty[i], (n - 1) & 1, abort_flag))) break;
+              // slot i's score columns are free once its softmax read the previous tile
+              if (g_t > 0 && !(ok = wait_bounded(&s_free[i], (g_t - 1) & 1, abort_flag))) break;
               tc_fence_after();
-              issue_pv(i, t > 1);
+              issue_s(i, g_t & 1);
+              umma_commit_pair(&s_full[i], kBoth);
+            }
+            if (!ok) break;
+            umma_commit_pair(&k_empty[g_t & 1], kBoth);
+            if (t == it.n_kt - 1) umma_commit_pair(q_empty, kBoth);
+          }
+          kt += it.n_kt;
+          ++n;
+        }
+      } else {
+        constexpr uint32_t idesc_o = idesc_bf16_f32(256, 128, false, true);
+        const uint32_t dP0 = desc_lo_sw128(sbase + kPpOffP, 16);
+        const uint32_t dV = desc_lo_sw128(sbase + kPpOffV, 16384);  // MN-major, one 64-column atom per CTA
+        // O_i += P_i V: 8 K-steps of 16 keys (A boxes 16 KB apart; B: 16 key rows = 2 KB)
+        auto issue_pv = [&](int i, bool acc) {
+          const uint32_t a = dP0 + static_cast<uint32_t>(i) * (kPpPBytes >> 4);
+          const uint32_t d = tbase + 256 + static_cast<uint32_t>(i) * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss_lo_pair(d, a + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
+                            dV + ((kk * 2048) >> 4), dhi, idesc_o, (acc || kk > 0) ? 1u : 0u);
+        };
+        int n = 0, kt = 0;
+        bool ok = true;
+        for (int r = 0; ok && r < rounds; ++r) {
+          const int item = pf_item_index(r, cl, nclusters);
+          if (item >= p.num_items) continue;
+          const PpItem it = pp_decode(p, item);
+          if (!it.valid) continue;
+          for (int t = 0; ok && t < it.n_kt; ++t) {
+            const int g_t = kt + t;
+            if (!(ok = wait_bounded(v_full, g_t & 1, abort_flag))) break;
+#pragma unroll 1
+            for (int i = 0; i < 2; ++i) {
+              if (!(ok = wait_bounded(&p_full[i], g_t & 1, abort_flag))) break;
+              // an item's first P.V overwrites O: the previous item's epilogue must have read it
+              if (t == 0 && n > 0 && !(ok = wait_bounded(&o_empty[i], (n - 1) & 1, abort_flag))) break;
+              tc_fence_after();
+              issue_pv(i, t > 0);
               umma_commit_pair(&pv_done[i], kBoth);
             }
             if (!ok) break;
             umma_commit_pair(v_empty, kBoth);
           }
+          kt += it.n_kt;
+          ++n;
         }
-        if (!ok) break;
-        // the item's last P.V
-        {
-          const int g_p = kt + it.n_kt - 1;
-          if (!(ok = wait_bounded(v_full, g_p & 1, abort_flag))) break;
-#pragma unroll 1
-          for (int i = 0; i < 2; ++i) {
-            if (!(ok = wait_bounded_cluster(&p_full[i], g_p & 1, abort_flag))) break;
-            if (it.n_kt == 1 && n > 0 && !(ok = wait_bounded_cluster(&o_empty[i], (n - 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(i, it.n_kt > 1);
-            umma_commit_pair(&pv_done[i], kBoth);
-          }
-          if (!ok) break;
-          umma_commit_pair(v_empty, kBoth);
-        }
-        kt += it.n_kt;
-        ++n;
       }
     }
   } else if (warp < 8) {
