@@ -28,8 +28,9 @@
 // warpgroup gives back down to 120 and the two softmax warpgroups take 192
 // (2*128*192 + 128*120 = 64512 = 384*168).
 //
-// Shared memory per CTA: Q_0, Q_1 (48 KB each), P_0, P_1 (32 KB each), K half
-// tiles in two stages (24 KB each), V half tile (16 KB).  TMEM per CTA:
+// Shared memory per CTA: Q_0, Q_1 (48 KB each), P_0, P_1 (32 KB each), the K
+// half tile (24 KB, one stage: the score stream has slack for its load),
+// V half tiles in two stages (16 KB each: the P.V stream has none).  TMEM per CTA:
 // S_0 [0,128)  S_1 [128,256)  O_0 [256,384)  O_1 [384,512).
 //
 // Barriers: loads are counted on the leader's full barriers (the leader's
@@ -54,9 +55,9 @@ constexpr int kPpKBytes = 64 * 192 * 2;         // 3 boxes of [64 keys][64 dims]
 constexpr int kPpVBytes = 128 * 64 * 2;         // 1 box of [128 keys][64 dims]
 constexpr int kPpOffQ = 0;                      // Q_0, Q_1
 constexpr int kPpOffP = 2 * kPpQBytes;          // 98304: P_0, P_1
-constexpr int kPpOffK = kPpOffP + 2 * kPpPBytes;  // 163840: 2 stages
-constexpr int kPpOffV = kPpOffK + 2 * kPpKBytes;  // 212992
-constexpr int kPpOffBar = kPpOffV + kPpVBytes;    // 229376
+constexpr int kPpOffK = kPpOffP + 2 * kPpPBytes;  // 163840: one stage
+constexpr int kPpOffV = kPpOffK + kPpKBytes;      // 188416: 2 stages
+constexpr int kPpOffBar = kPpOffV + 2 * kPpVBytes;  // 221184
 constexpr int kPpSmemBytes = kPpOffBar + 256 + 1024;
 
 struct PairParams {
@@ -115,15 +116,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPpOffBar);
   // leader-side (arrivals / bytes of both CTAs counted there)
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = bars + 2;    // [2]
   uint64_t* s_free = bars + 4;    // [2] slot i's softmax of both CTAs read S_i
   uint64_t* p_full = bars + 6;    // [2] slot i's P tiles of both CTAs written
   uint64_t* o_empty = bars + 8;   // [2] slot i's O read by both epilogues
   // both CTAs (MMA completions, committed with CTA mask 0b11)
   uint64_t* q_empty = bars + 10;
-  uint64_t* k_empty = bars + 11;  // [2]
-  uint64_t* v_empty = bars + 13;
+  uint64_t* k_empty = bars + 11;
+  uint64_t* v_empty = bars + 12;  // [2]
   uint64_t* s_full = bars + 14;   // [2]
   uint64_t* pv_done = bars + 16;  // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
@@ -137,12 +138,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
   if (warp == 8) {
     if (lane == 0) {
       mbar_init(q_full, 1);
-      mbar_init(v_full, 1);
+      mbar_init(k_full, 1);
       mbar_init(q_empty, 1);
-      mbar_init(v_empty, 1);
+      mbar_init(k_empty, 1);
       for (int i = 0; i < 2; ++i) {
-        mbar_init(&k_full[i], 1);
-        mbar_init(&k_empty[i], 1);
+        mbar_init(&v_full[i], 1);
+        mbar_init(&v_empty[i], 1);
         mbar_init(&s_free[i], 8);   // one elected lane per softmax warp of both CTAs
         mbar_init(&p_full[i], 8);   // one elected lane per softmax warp of both CTAs
         mbar_init(&o_empty[i], 8);   // one elected lane per softmax warp of both CTAs
@@ -184,7 +185,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
     // never holds back the next key tile's K.
     if (lane == 0) {
       tma_prefetch_desc(&tm_v);
-      const uint32_t bv = lead(v_full);
+      const uint32_t bv0 = lead(&v_full[0]), bv1 = lead(&v_full[1]);
       int kt = 0;
       bool ok = true;
       for (int r = 0; ok && r < rounds; ++r) {
@@ -193,9 +194,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
         const PpItem it = pp_decode(p, item);
         if (!it.valid) continue;
         for (int t = 0; t < it.n_kt; ++t, ++kt) {
-          if (kt >= 1 && !(ok = wait_bounded(v_empty, (kt - 1) & 1, abort_flag))) break;
-          if (rank == 0) mbar_arrive_expect_tx(v_full, 2 * kPpVBytes);
-          tma_load_3d_pair(smem + kPpOffV, &tm_v, bv, 64 * (int)rank, it.g, it.b0 + (it.j_lo + t) * kPfTile);
+          const int vs = kt & 1;
+          if (kt >= 2 && !(ok = wait_bounded(&v_empty[vs], ((kt >> 1) - 1) & 1, abort_flag))) break;
+          if (rank == 0) mbar_arrive_expect_tx(&v_full[vs], 2 * kPpVBytes);
+          tma_load_3d_pair(smem + kPpOffV + vs * kPpVBytes, &tm_v, vs ? bv1 : bv0, 64 * (int)rank, it.g,
+                           it.b0 + (it.j_lo + t) * kPfTile);
         }
       }
     }
@@ -204,7 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
-      const uint32_t bq = lead(q_full), bk0 = lead(&k_full[0]), bk1 = lead(&k_full[1]);
+      const uint32_t bq = lead(q_full), bk = lead(k_full);
       int n = 0, kt = 0;
       bool ok = true;
       for (int r = 0; ok && r < rounds; ++r) {
@@ -235,14 +238,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           break;
         }
         for (int t = 0; t < it.n_kt; ++t, ++kt) {
-          const int ks = kt & 1;
           const int row = it.b0 + (it.j_lo + t) * kPfTile;
-          if (kt >= 2 && !(ok = wait_bounded(&k_empty[ks], ((kt >> 1) - 1) & 1, abort_flag))) break;
-          if (rank == 0) mbar_arrive_expect_tx(&k_full[ks], 2 * kPpKBytes);
+          if (kt >= 1 && !(ok = wait_bounded(k_empty, (kt - 1) & 1, abort_flag))) break;
+          if (rank == 0) mbar_arrive_expect_tx(k_full, 2 * kPpKBytes);
 #pragma unroll
           for (int c = 0; c < 3; ++c)
-            tma_load_3d_pair(smem + kPpOffK + ks * kPpKBytes + c * 8192, &tm_k, ks ? bk1 : bk0, c * 64,
-                             it.g, row + 64 * (int)rank);
+            tma_load_3d_pair(smem + kPpOffK + c * 8192, &tm_k, bk, c * 64, it.g, row + 64 * (int)rank);
         }
         ++n;
       }
@@ -261,9 +262,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
         const uint32_t dQ0 = desc_lo_sw128(sbase + kPpOffQ, 16);
         const uint32_t dK0 = desc_lo_sw128(sbase + kPpOffK, 16);
         // S_i = Q_i K^T: 12 K-steps of 16 dims (A boxes 16 KB apart, B boxes 8 KB apart)
-        auto issue_s = [&](int i, int ks) {
+        auto issue_s = [&](int i) {
           const uint32_t a = dQ0 + static_cast<uint32_t>(i) * (kPpQBytes >> 4);
-          const uint32_t b = dK0 + static_cast<uint32_t>(ks) * (kPpKBytes >> 4);
+          const uint32_t b = dK0;
           const uint32_t d = tbase + static_cast<uint32_t>(i) * 128;
 #pragma unroll
           for (int kk = 0; kk < 12; ++kk)
@@ -280,17 +281,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           if (!(ok = wait_bounded(q_full, n & 1, abort_flag))) break;
           for (int t = 0; ok && t < it.n_kt; ++t) {
             const int g_t = kt + t;  // tile index over all items
-            if (!(ok = wait_bounded(&k_full[g_t & 1], (g_t >> 1) & 1, abort_flag))) break;
+            if (!(ok = wait_bounded(k_full, g_t & 1, abort_flag))) break;
 #pragma unroll 1
             for (int i = 0; i < 2; ++i) {
               // slot i's score columns are free once its softmax read the previous tile
               if (g_t > 0 && !(ok = wait_bounded(&s_free[i], (g_t - 1) & 1, abort_flag))) break;
               tc_fence_after();
-              issue_s(i, g_t & 1);
+              issue_s(i);
               umma_commit_pair(&s_full[i], kBoth);
             }
             if (!ok) break;
-            umma_commit_pair(&k_empty[g_t & 1], kBoth);
+            umma_commit_pair(k_empty, kBoth);
             if (t == it.n_kt - 1) umma_commit_pair(q_empty, kBoth);
           }
           kt += it.n_kt;
@@ -299,15 +300,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
       } else {
         constexpr uint32_t idesc_o = idesc_bf16_f32(256, 128, false, true);
         const uint32_t dP0 = desc_lo_sw128(sbase + kPpOffP, 16);
-        const uint32_t dV = desc_lo_sw128(sbase + kPpOffV, 16384);  // MN-major, one 64-column atom per CTA
+        const uint32_t dV0 = desc_lo_sw128(sbase + kPpOffV, 16384);  // MN-major, one 64-column atom per CTA
         // O_i += P_i V: 8 K-steps of 16 keys (A boxes 16 KB apart; B: 16 key rows = 2 KB)
-        auto issue_pv = [&](int i, bool acc) {
+        auto issue_pv = [&](int i, int vs, bool acc) {
           const uint32_t a = dP0 + static_cast<uint32_t>(i) * (kPpPBytes >> 4);
           const uint32_t d = tbase + 256 + static_cast<uint32_t>(i) * 128;
+          const uint32_t bv = dV0 + static_cast<uint32_t>(vs) * (kPpVBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_ss_lo_pair(d, a + ((((kk >> 2) * 16384) + (kk & 3) * 32) >> 4),
-                            dV + ((kk * 2048) >> 4), dhi, idesc_o, (acc || kk > 0) ? 1u : 0u);
+                            bv + ((kk * 2048) >> 4), dhi, idesc_o, (acc || kk > 0) ? 1u : 0u);
         };
         int n = 0, kt = 0;
         bool ok = true;
@@ -318,18 +320,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           if (!it.valid) continue;
           for (int t = 0; ok && t < it.n_kt; ++t) {
             const int g_t = kt + t;
-            if (!(ok = wait_bounded(v_full, g_t & 1, abort_flag))) break;
+            if (!(ok = wait_bounded(&v_full[g_t & 1], (g_t >> 1) & 1, abort_flag))) break;
 #pragma unroll 1
             for (int i = 0; i < 2; ++i) {
               if (!(ok = wait_bounded(&p_full[i], g_t & 1, abort_flag))) break;
               // an item's first P.V overwrites O: the previous item's epilogue must have read it
               if (t == 0 && n > 0 && !(ok = wait_bounded(&o_empty[i], (n - 1) & 1, abort_flag))) break;
               tc_fence_after();
-              issue_pv(i, t > 0);
+              issue_pv(i, g_t & 1, t > 0);
               umma_commit_pair(&pv_done[i], kBoth);
             }
             if (!ok) break;
-            umma_commit_pair(v_empty, kBoth);
+            umma_commit_pair(&v_empty[g_t & 1], kBoth);
           }
           kt += it.n_kt;
           ++n;

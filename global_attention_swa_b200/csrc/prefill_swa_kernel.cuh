@@ -26,7 +26,12 @@
 //               window skip the per-element mask.
 //   warps 8-11  epilogue: O / l -> bf16/fp32 rows, lse.
 //
-// TMEM: S_0 [0, 192), S_1 [192, 384), O [384, 512).
+// The output is normalised by the sum of the bf16-rounded P that P.V
+// multiplies (plus the sink's term): a second small MMA per key step,
+// P x (a 16-column block of ones), accumulates exactly that row sum in TMEM,
+// so the softmax warps keep only the unrounded sum (for lse).
+//
+// TMEM: S_0 [0, 176), S_1 [176, 352), O [352, 480), rounded-P row sum [480, 496).
 #pragma once
 
 #include "common.cuh"
@@ -34,14 +39,17 @@
 namespace mimo {
 
 constexpr int kSwThreads = 448;
-constexpr int kSwNMax = 192;
+constexpr int kSwNMax = 176;
 constexpr int kSwQBytes = 3 * 16384;                   // [128 rows][192 dims] as 3 boxes
 constexpr int kSwKBox = kSwNMax * 128;                 // [N rows][64 dims], 1024-aligned
 constexpr int kSwOffQ = 0;                             // 2 buffers
 constexpr int kSwOffK = 2 * kSwQBytes;                 // 98304: 3 boxes
 constexpr int kSwOffV = kSwOffK + 3 * kSwKBox;         // 172032: 2 boxes
-constexpr int kSwOffML = kSwOffV + 2 * kSwKBox;        // 221184: [2][128] float2
-constexpr int kSwOffBar = kSwOffML + 2 * 128 * 8;      // 223232
+constexpr int kSwOffML = kSwOffV + 2 * kSwKBox;        // [2][128] float4 (m, l, sink term, -)
+constexpr int kSwOffOnes = kSwOffML + 2 * 128 * 16;    // [16 rows][64] bf16 ones, 1024-aligned
+constexpr int kSwOffBar = kSwOffOnes + 2048;
+constexpr uint32_t kSwColO = 2 * kSwNMax, kSwColSum = kSwColO + 128;  // 352, 480
+static_assert(kSwOffOnes % 1024 == 0 && kSwColSum + 16 <= 512, "SWA prefill layout");
 constexpr int kSwSmemBytes = kSwOffBar + 256 + 1024;
 
 struct SwaParams {
@@ -114,9 +122,13 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   uint64_t* ml_empty = bars + 16; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
-  float2* ml = reinterpret_cast<float2*>(smem + kSwOffML);  // [2][128] (output factor, lse) per row
+  float4* ml = reinterpret_cast<float4*>(smem + kSwOffML);  // [2][128] (m, l, sink term) per row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the ones block (B operand of the row-sum MMAs): 2 KB of bf16 1.0
+  for (int i = threadIdx.x; i < 2048 / 4; i += kSwThreads)
+    reinterpret_cast<uint32_t*>(smem + kSwOffOnes)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
   if (warp == 12) {
     if (lane == 0) {
       for (int i = 0; i < 2; ++i) {
@@ -162,10 +174,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
                       it.g * p.G, it.b0 + it.q0 + blk * p.QB);
       };
       // Blocks are numbered n = 0, 1, ... over this CTA's pairs; block n uses Q
-      // buffer n & 1.  The pair's K/V window is loaded at its first block.  The
-      // next pair's Q and K/V are prefetched into L2 when a pair starts, two
-      // blocks ahead of their loads (a Q tile from DRAM takes longer than one
-      // block's work, and there is no room for a third Q buffer).
+      // buffer n & 1.  The pair's K/V window is loaded at its first block.
       SwItem cur, nxt;
       int r = sw_next(p, 0, rounds, cur);
       if (r >= 0) load_q(cur, 0, 0);
@@ -181,17 +190,6 @@ __global__ void __launch_bounds__(kSwThreads, 1)
 #pragma unroll
             for (int c = 0; c < 3; ++c)
               tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
-            if (rn >= 0) {
-              const int nk0 = nxt.b0 + nxt.q0 + 2 * p.QB - N;
-#pragma unroll
-              for (int c = 0; c < 3; ++c) {
-                for (int b = 0; b < nxt.nblk; ++b)
-                  tma_prefetch_l2_3d(&tm_q, c * 64, nxt.g * p.G, nxt.b0 + nxt.q0 + b * p.QB);
-                tma_prefetch_l2_3d(&tm_k, c * 64, nxt.g, nk0);
-              }
-#pragma unroll
-              for (int c = 0; c < 2; ++c) tma_prefetch_l2_3d(&tm_v, c * 64, nxt.g, nk0);
-            }
           }
           // the next block's Q, one block ahead (its buffer was freed by S(n-1))
           const int bn = (n + 1) & 1;
@@ -221,7 +219,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, N, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t tO = tbase + 384;
+      const uint32_t tO = tbase + kSwColO, tSum = tbase + kSwColSum;
+      constexpr uint32_t idesc_sum = idesc_bf16_f32(128, 16, false, false);
+      // every K step reuses the same 16 x 16 block of ones (K-major, 128-byte rows)
+      const uint64_t ones_desc = smem_desc_sw128(sbase + kSwOffOnes, 16, 1024);
       bool ok = true;
       // O = P(m) V over N keys: N/16 MMAs (P: 8 TMEM columns each; V: 16 rows = 2 KB).
       // Block m is the blk-th of pair kp_m; the pair's V is waited for at its first
@@ -237,6 +238,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         for (int kk = 0; kk < N / 16; ++kk)
           umma_ts(tO, tP + kk * 8, smem_desc_sw128(aV + kk * 2048, kSwKBox, 1024), idesc_o,
                   kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < N / 16; ++kk)  // row sums of the same P
+          umma_ts(tSum, tP + kk * 8, ones_desc, idesc_sum, kk > 0 ? 1u : 0u);
         umma_commit(o_full);
         if (last_of_pair) umma_commit(v_empty);
       };
@@ -323,9 +326,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       // pass 2: P = 2^(s*scale - m) (0 outside the window), bf16 over the same
       // columns (P of columns [c0, c0 + 48) lands in [c0 / 2, c0 / 2 + 24), behind
-      // the read position).  The unrounded sum gives lse; the sum of the rounded
-      // P (the values P.V multiplies) normalises the output.
-      float2 l2 = make_float2(0.f, 0.f), lr2 = make_float2(0.f, 0.f);
+      // the read position).  The unrounded sum gives lse; the output's
+      // normaliser, the sum of the rounded P, comes from the row-sum MMA.
+      float2 l2 = make_float2(0.f, 0.f);
       for (int c0 = 0; c0 < N; c0 += 48) {
         uint32_t v[48];
         tmem_load48_sync(tS + c0, v);
@@ -341,7 +344,6 @@ __global__ void __launch_bounds__(kSwThreads, 1)
               const float2 pe = make_float2(ex2(x.x), ex2(x.y));
               pk[e] = pack_bf16(pe.x, pe.y);
               l2 = add2(l2, pe);
-              lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
             }
           } else {
 #pragma unroll
@@ -353,7 +355,6 @@ __global__ void __launch_bounds__(kSwThreads, 1)
                                             (c + 1 >= c_lo && c + 1 <= c_hi) ? ex2(x1) : 0.f);
               pk[e] = pack_bf16(pe.x, pe.y);
               l2 = add2(l2, pe);
-              lr2 = add2(lr2, make_float2(bf16_lo(pk[e]), bf16_hi(pk[e])));
             }
           }
           if (cq0 < N) tmem_st8(tS + cq0 / 2, pk);
@@ -362,16 +363,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
-      float l = l2.x + l2.y, lr = lr2.x + lr2.y;
-      if (p.sinks && m != -INFINITY) {
-        const float ps = ex2(sg2 - m);
-        l += ps;
-        lr += ps;
-      }
-      const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
-      const float lse = (l > 0.f) ? (m * 0.6931471805599453f + logf(l)) : -INFINITY;
+      const float ps = (p.sinks && m != -INFINITY) ? ex2(sg2 - m) : 0.f;  // the sink's term
       if (n >= 2 && !(ok = wait_bounded(&ml_empty[b], ((n >> 1) - 1) & 1, abort_flag))) break;
-      ml[b * 128 + r] = make_float2(f, lse);
+      ml[b * 128 + r] = make_float4(m, l2.x + l2.y + ps, ps, 0.f);
       mbar_arrive(&ml_full[b]);
     }
   } else if (warp < 12) {
@@ -379,7 +373,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     const int r = threadIdx.x - 256;
     const int a = r / p.G, hh = r % p.G;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tO = tbase + lane_off + 384;
+    const uint32_t tO = tbase + lane_off + kSwColO;
     SwItem it;
     int n = 0;
     bool ok = true;
@@ -389,13 +383,16 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       if (!(ok = wait_bounded(o_full, n & 1, abort_flag))) break;
       tc_fence_after();
       if (!(ok = wait_bounded(&ml_full[b], (n >> 1) & 1, abort_flag))) break;
-      const float2 mlv = ml[b * 128 + r];
+      const float4 mlv = ml[b * 128 + r];  // m (base 2), unrounded sum with the sink, the sink's term
       mbar_arrive(&ml_empty[b]);
+      float rs[16];
+      tmem_load16_sync(tbase + lane_off + kSwColSum, rs);  // rounded-P row sum (16 equal columns)
+      const float lr = rs[0] + mlv.z;
       const int qpos = it.q0 + blk * p.QB + a;
       const bool live = qpos < it.len;
       const int tok = it.b0 + qpos;
       const int hg = it.g * p.G + hh;
-      const float f = mlv.x;
+      const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
       const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
       // O in two 64-column halves (registers: 448 threads leave 128 per thread);
       // O is released to the next P.V after the second half is in registers.
@@ -449,7 +446,9 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           }
         }
       }
-      if (live && p.lse) p.lse[(size_t)hg * p.total + tok] = mlv.y;
+      if (live && p.lse)
+        p.lse[(size_t)hg * p.total + tok] =
+            (mlv.y > 0.f) ? (mlv.x * 0.6931471805599453f + logf(mlv.y)) : -INFINITY;
     }
   }
 
