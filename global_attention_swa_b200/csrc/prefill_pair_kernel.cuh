@@ -223,20 +223,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
           for (int c = 0; c < 3; ++c)
             tma_load_3d_pair(smem + kPpOffQ + s * kPpQBytes + c * 16384, &tm_q, bq, c * 64,
                              it.h0 + 2 * (int)rank + s, it.b0 + it.q0);
-        // the next item's Q into L2 now, so that its load (after this item's
-        // last score tile) does not wait for DRAM
-        for (int r2 = r + 1; r2 < rounds; ++r2) {
-          const int item2 = pf_item_index(r2, cl, nclusters);
-          if (item2 >= p.num_items) continue;
-          const PpItem nx = pp_decode(p, item2);
-          if (!nx.valid) continue;
-#pragma unroll
-          for (int s = 0; s < 2; ++s)
-#pragma unroll
-            for (int c = 0; c < 3; ++c)
-              tma_prefetch_l2_3d(&tm_q, c * 64, nx.h0 + 2 * (int)rank + s, nx.b0 + nx.q0);
-          break;
-        }
         for (int t = 0; t < it.n_kt; ++t, ++kt) {
           const int row = it.b0 + (it.j_lo + t) * kPfTile;
           if (kt >= 1 && !(ok = wait_bounded(k_empty, (kt - 1) & 1, abort_flag))) break;
@@ -244,6 +230,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPpThreads, 1)
 #pragma unroll
           for (int c = 0; c < 3; ++c)
             tma_load_3d_pair(smem + kPpOffK + c * 8192, &tm_k, bk, c * 64, it.g, row + 64 * (int)rank);
+          if (t == 0) {
+            // with the item's first loads out, bring the next item's Q into L2,
+            // so that its load after this item's last score tile skips DRAM
+            for (int r2 = r + 1; r2 < rounds; ++r2) {
+              const int item2 = pf_item_index(r2, cl, nclusters);
+              if (item2 >= p.num_items) continue;
+              const PpItem nx = pp_decode(p, item2);
+              if (!nx.valid) continue;
+#pragma unroll
+              for (int s = 0; s < 2; ++s)
+#pragma unroll
+                for (int c = 0; c < 3; ++c)
+                  tma_prefetch_l2_3d(&tm_q, c * 64, nx.h0 + 2 * (int)rank + s, nx.b0 + nx.q0);
+              break;
+            }
+          }
         }
         ++n;
       }

@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       int n = 0, kp = 0;
       while (ok && r >= 0) {
         const int k0 = cur.q0 + 2 * p.QB - N;  // may be negative: zero-filled or masked
-        const int rn = sw_next(p, r + 1, rounds, nxt);
+        int rn = -1;
         for (int blk = 0; ok && blk < cur.nblk; ++blk, ++n) {
           if (blk == 0) {
             if (kp >= 1 && !(ok = wait_bounded(k_empty, (kp - 1) & 1, abort_flag))) break;
@@ -191,9 +191,11 @@ __global__ void __launch_bounds__(kSwThreads, 1)
             for (int c = 0; c < 3; ++c)
               tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
           }
-          // the next block's Q, one block ahead (its buffer was freed by S(n-1))
+          // the next block's Q, one block ahead (its buffer was freed by S(n-1));
+          // the next pair is looked up only now, after this pair's loads are out
           const int bn = (n + 1) & 1;
           const bool next_in_pair = (blk + 1 < cur.nblk);
+          if (!next_in_pair) rn = sw_next(p, r + 1, rounds, nxt);
           if (next_in_pair || rn >= 0) {
             if (n + 1 >= 2 && !(ok = wait_bounded(&q_empty[bn], (((n + 1) >> 1) - 1) & 1, abort_flag))) break;
             if (next_in_pair)
