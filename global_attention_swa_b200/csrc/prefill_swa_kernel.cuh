@@ -27,11 +27,12 @@
 //   warps 8-11  epilogue: O / l -> bf16/fp32 rows, lse.
 //
 // The output is normalised by the sum of the bf16-rounded P that P.V
-// multiplies (plus the sink's term): a second small MMA per key step,
-// P x (a 16-column block of ones), accumulates exactly that row sum in TMEM,
-// so the softmax warps keep only the unrounded sum (for lse).
+// multiplies (plus the sink's term).  The value operand of P.V carries a third
+// 64-column block that holds ones, and the product runs with N = 144: O's
+// columns 128..143 then accumulate exactly that row sum, at no extra MMA
+// instruction, and the softmax warps keep only the unrounded sum (for lse).
 //
-// TMEM: S_0 [0, 176), S_1 [176, 352), O [352, 480), rounded-P row sum [480, 496).
+// TMEM: S_0 [0, 160), S_1 [160, 320), O [320, 448) + rounded-P row sum [448, 464).
 #pragma once
 
 #include "common.cuh"
@@ -39,16 +40,16 @@
 namespace mimo {
 
 constexpr int kSwThreads = 448;
-constexpr int kSwNMax = 176;
+constexpr int kSwNMax = 160;
 constexpr int kSwQBytes = 3 * 16384;                   // [128 rows][192 dims] as 3 boxes
 constexpr int kSwKBox = kSwNMax * 128;                 // [N rows][64 dims], 1024-aligned
 constexpr int kSwOffQ = 0;                             // 2 buffers
 constexpr int kSwOffK = 2 * kSwQBytes;                 // 98304: 3 boxes
-constexpr int kSwOffV = kSwOffK + 3 * kSwKBox;         // 172032: 2 boxes
-constexpr int kSwOffML = kSwOffV + 2 * kSwKBox;        // [2][128] float4 (m, l, sink term, -)
-constexpr int kSwOffOnes = kSwOffML + 2 * 128 * 16;    // [16 rows][64] bf16 ones, 1024-aligned
-constexpr int kSwOffBar = kSwOffOnes + 2048;
-constexpr uint32_t kSwColO = 2 * kSwNMax, kSwColSum = kSwColO + 128;  // 352, 480
+constexpr int kSwOffV = kSwOffK + 3 * kSwKBox;         // 2 boxes
+constexpr int kSwOffOnes = kSwOffV + 2 * kSwKBox;      // the third value block: [N rows][64] ones
+constexpr int kSwOffML = kSwOffOnes + kSwKBox;          // [2][128] float4 (m, l, sink term, -)
+constexpr int kSwOffBar = kSwOffML + 2 * 128 * 16;
+constexpr uint32_t kSwColO = 2 * kSwNMax, kSwColSum = kSwColO + 128;  // 320, 448
 static_assert(kSwOffOnes % 1024 == 0 && kSwColSum + 16 <= 512, "SWA prefill layout");
 constexpr int kSwSmemBytes = kSwOffBar + 256 + 1024;
 
@@ -125,8 +126,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   float4* ml = reinterpret_cast<float4*>(smem + kSwOffML);  // [2][128] (m, l, sink term) per row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the ones block (B operand of the row-sum MMAs): 2 KB of bf16 1.0
-  for (int i = threadIdx.x; i < 2048 / 4; i += kSwThreads)
+  // the ones block, third 64-column block of the value operand: bf16 1.0
+  for (int i = threadIdx.x; i < kSwKBox / 4; i += kSwThreads)
     reinterpret_cast<uint32_t*>(smem + kSwOffOnes)[i] = 0x3F803F80u;
   fence_proxy_async_smem();
   if (warp == 12) {
@@ -220,11 +221,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, N, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
-      const uint32_t tO = tbase + kSwColO, tSum = tbase + kSwColSum;
-      constexpr uint32_t idesc_sum = idesc_bf16_f32(128, 16, false, false);
-      // every K step reuses the same 16 x 16 block of ones (K-major, 128-byte rows)
-      const uint64_t ones_desc = smem_desc_sw128(sbase + kSwOffOnes, 16, 1024);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 144, false, true);  // 128 value dims + 16 ones
+      const uint32_t tO = tbase + kSwColO;
       bool ok = true;
       // O = P(m) V over N keys: N/16 MMAs (P: 8 TMEM columns each; V: 16 rows = 2 KB).
       // Block m is the blk-th of pair kp_m; the pair's V is waited for at its first
@@ -240,8 +238,6 @@ __global__ void __launch_bounds__(kSwThreads, 1)
         for (int kk = 0; kk < N / 16; ++kk)
           umma_ts(tO, tP + kk * 8, smem_desc_sw128(aV + kk * 2048, kSwKBox, 1024), idesc_o,
                   kk > 0 ? 1u : 0u);
-        for (int kk = 0; kk < N / 16; ++kk)  // row sums of the same P
-          umma_ts(tSum, tP + kk * 8, ones_desc, idesc_sum, kk > 0 ? 1u : 0u);
         umma_commit(o_full);
         if (last_of_pair) umma_commit(v_empty);
       };
