@@ -12,7 +12,7 @@ LIB = os.path.join(PKG, "libmimo_attn.so")
 DEPS = [
     os.path.join(PKG, "csrc", f)
     for f in ("mimo_attn.cu", "common.cuh", "decode_kernel.cuh", "prefill_kernel.cuh",
-              "prefill_swa_kernel.cuh", "prefill_pair_kernel.cuh", "decode_fp8_kernel.cuh",
+              "prefill_swa_kernel.cuh", "decode_fp8_kernel.cuh",
               "rope_append_kernel.cuh", "decode_merge_kernel.cuh",
               "backward_kernel.cuh", "backward_tc_kernel.cuh", "backward_dq_tc_kernel.cuh")
 ] + [os.path.join(ROOT, "include", "mimo_attn.h")]

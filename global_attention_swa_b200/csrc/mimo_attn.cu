@@ -22,7 +22,6 @@
 #include "backward_dq_tc_kernel.cuh"
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
-#include "prefill_pair_kernel.cuh"
 
 namespace {
 
@@ -136,11 +135,6 @@ mimo_status_t ensure_attributes() {
                                             mimo::kPfSmemBytes),
                        "prefill smem attribute")))
     return st;
-  if ((st = cuda_check(cudaFuncSetAttribute(mimo::prefill_pair_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            mimo::kPpSmemBytes),
-                       "pair prefill smem attribute")))
-    return st;
   if ((st = cuda_check(cudaFuncSetAttribute(mimo::prefill_swa_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             mimo::kSwSmemBytes),
@@ -205,32 +199,6 @@ int sm_count() {
   if (c <= 0) {
     if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
       c = 148;
-    counts[dev].store(c, std::memory_order_relaxed);
-  }
-  return c;
-}
-
-// Clusters of two CTAs of the pair prefill that fit on the current device at
-// once (74 on B200: one CTA per SM); the persistent grid is sized to it.
-int pair_clusters() {
-  static std::atomic<int> counts[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
-  int c = counts[dev].load(std::memory_order_relaxed);
-  if (c <= 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
-    cfg.blockDim = dim3(mimo::kPpThreads, 1, 1);
-    cfg.dynamicSmemBytes = mimo::kPpSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&c, (void*)mimo::prefill_pair_kernel, &cfg) != cudaSuccess || c <= 0)
-      c = sm_count() / 2;
     counts[dev].store(c, std::memory_order_relaxed);
   }
   return c;
@@ -365,9 +333,6 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
     return ok();
   }
 
-  // Query heads in groups of four per key/value head: CTA pairs (M = 256 MMAs),
-  // each CTA holding two heads and half of every K / V tile.
-  const bool pair = (G % 4) == 0;
   CUtensorMap tq, tk, tv;
   {
     const uint64_t d[3] = {192, (uint64_t)Hq, (uint64_t)total_tokens};
@@ -378,43 +343,14 @@ mimo_status_t mimo_attn_prefill(const mimo_attn_dims_t* dims, const void* q, con
   {
     const uint64_t d[3] = {192, (uint64_t)Hkv, (uint64_t)total_tokens};
     const uint64_t s[2] = {192 * 2, (uint64_t)Hkv * 192 * 2};
-    const uint32_t b[3] = {64, 1, pair ? 64u : 128u};  // pairs: each CTA loads 64 of the 128 keys
+    const uint32_t b[3] = {64, 1, 128};
     if ((st = make_map(&tk, k, 3, d, s, b))) return st;
   }
   {
     const uint64_t d[3] = {128, (uint64_t)Hkv, (uint64_t)total_tokens};
     const uint64_t s[2] = {128 * 2, (uint64_t)Hkv * 128 * 2};
-    const uint32_t b[3] = {64, 1, 128};  // pairs: each CTA loads one of the two 64-dim boxes
+    const uint32_t b[3] = {64, 1, 128};
     if ((st = make_map(&tv, v, 3, d, s, b))) return st;
-  }
-  if (pair) {
-    mimo::PairParams pp;
-    pp.cu_seqlens = cu_seqlens;
-    pp.sinks = sinks;
-    pp.out = out;
-    pp.lse = lse;
-    pp.total = total_tokens;
-    pp.Hq = Hq;
-    pp.Hkv = Hkv;
-    pp.G = G;
-    pp.window = window;
-    pp.quads_per_group = G / 4;
-    pp.num_seqs = num_seqs;
-    pp.max_seqlen = max_seqlen;
-    pp.num_qtiles = (max_seqlen + mimo::kPfTile - 1) / mimo::kPfTile;
-    const long items = (long)pp.num_qtiles * Hkv * pp.quads_per_group * num_seqs;
-    if (items > 0x7fffffffL) return fail(MIMO_ERR_UNSUPPORTED, "too many work items (%ld)", items);
-    pp.num_items = (int)items;
-    pp.scale_log2 = scale_log2_of(dims);
-    pp.v_scale = v_scale_of(dims);
-    pp.out_f32 = dims->out_dtype == MIMO_DTYPE_F32;
-    pp.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
-    // persistent: one pair of CTAs per two SMs
-    const int clusters = (int)std::min<long>(items, std::max(1, pair_clusters()));
-    mimo::prefill_pair_kernel<<<2 * clusters, mimo::kPpThreads, mimo::kPpSmemBytes, (cudaStream_t)stream>>>(
-        tq, tk, tv, pp);
-    if ((st = cuda_check(cudaGetLastError(), "pair prefill launch"))) return st;
-    return ok();
   }
   mimo::PrefillParams p;
   p.cu_seqlens = cu_seqlens;

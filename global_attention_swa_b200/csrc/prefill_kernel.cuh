@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float2 e = make_float2(ex2(x.x), ex2(x.y));
             pk[c] = pack_bf16(e.x, e.y);
             acc[c & 1] = add2(acc[c & 1], e);
-            acr[c & 1] = add2(acr[c & 1], make_float2(bf16_lo(pk[c]), bf16_hi(pk[c])));
+            add_bf16x2(acr[c & 1], pk[c]);
           }
           tmem_st32(tS + 32 * half, pk);
         }

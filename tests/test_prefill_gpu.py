@@ -60,31 +60,31 @@ def test_varlen_pack_with_empty_and_single_token_sequences(window):
     P.check(out, ro, lse, rl, what=f"varlen W={window}")
 
 
-# query heads in groups of four per key/value head run on CTA pairs (M = 256
-# MMAs, two heads per CTA); groups of 8 with a window the packed kernel cannot
-# hold (N > 192), and groups of 4 with any window, take the pair kernel too
+# global layers (window 0) and windows the packed sliding-window kernel cannot
+# hold (N > 160) run on the per-head kernel: every length class around the
+# 128-row tile edge, at several head groupings
 
 
 @pytest.mark.parametrize("hq,hkv,window", [(8, 2, 0), (8, 2, 1), (8, 2, 2), (8, 2, 129),
                                            (32, 2, 0), (32, 4, 300), (4, 1, 128)])
-def test_pair_kernel_lengths(hq, hkv, window):
+def test_per_head_kernel_lengths(hq, hkv, window):
     for T in (1, 2, 127, 128, 129, 255, 256, 257, 1000):
         sinks = (T + window) % 2 == 1
         x = W.prefill_inputs([T], hq=hq, hkv=hkv, seed=T * 13 + window + hq, sinks=sinks)
         out_dtype = torch.bfloat16 if T % 3 == 0 else torch.float32
         out, lse = run_gpu(x, window, out_dtype)
         ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
-        P.check(out, ro, lse, rl, what=f"pair Hq={hq} Hkv={hkv} T={T} W={window}")
+        P.check(out, ro, lse, rl, what=f"per-head Hq={hq} Hkv={hkv} T={T} W={window}")
 
 
-def test_pair_kernel_many_items_per_cluster_varlen():
-    """More items than CTA pairs, with sequences of every length class packed."""
+def test_per_head_kernel_varlen_every_length_class():
+    """Sequences of every length class packed into one call."""
     lengths = [1, 1000, 0, 129, 2000, 127, 3, 700, 128, 1500]
     x = W.prefill_inputs(lengths, hq=16, hkv=2, seed=61)
     for window in (0, 500):
         out, lse = run_gpu(x, window, torch.float32)
         ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
-        P.check(out, ro, lse, rl, what=f"pair varlen W={window}")
+        P.check(out, ro, lse, rl, what=f"per-head varlen W={window}")
 
 
 def test_varlen_pack_equals_separate_calls():
@@ -217,12 +217,13 @@ def test_output_only_16_byte_aligned(odt):
 
 # ----------------------------------------------------------------------------
 # sliding window with the key/value group packed into the MMA rows
-# (G = Hq/Hkv in {8, 16, 32}; N = roundup16(W + 128/G - 1) <= 192, else the
-# general kernel takes the call)
+# (G = Hq/Hkv in {8, 16, 32}; N = roundup16(W + 128/G - 1) <= 160, else the
+# per-head kernel takes the call: the largest packed windows are 129 at G=8,
+# 145 at G=16 and 153 at G=32, and the next window up crosses to the other kernel)
 
 
 @pytest.mark.parametrize("hq,hkv", [(16, 1), (16, 2), (64, 2)])
-@pytest.mark.parametrize("window", [1, 2, 8, 128, 129, 130, 177, 185, 186])
+@pytest.mark.parametrize("window", [1, 2, 8, 128, 129, 130, 145, 146, 153, 154, 186])
 def test_packed_window_lengths(hq, hkv, window):
     for T in (1, 2, 7, 8, 9, 127, 129, 300, 1000):
         sinks = (T + window) % 3 != 0
