@@ -33,10 +33,14 @@
 //
 // Online softmax in base 2 with the sink folded into the running state:
 // m starts at sigma_h*log2(e) and l at 1 (the sink's own term), so the sink
-// enters the normaliser once and never the output.  The running max is only
-// moved (and O rescaled) when a row's max grows by more than kRescaleLog2;
-// otherwise P is computed against the stale max (P <= 2^kRescaleLog2), which
-// is exact because O and l share the same reference.
+// enters the normaliser once and never the output.  The reference m is not
+// the running max: P = 2^(s*scale - m) is computed against it as it stands,
+// and it is moved to the row max (with O and l rescaled) only when a tile's
+// sum of P leaves the range where fp32 and bf16 hold it (above 2^64, or NaN
+// from an overflow), or a row without a sink has no reference yet.  That is
+// exact, because O and l share the reference, and the relative precision of
+// bf16 P and of the fp32 sums does not depend on their scale.  The common
+// path therefore does no row-max pass at all.
 //
 // Key tiles wholly outside [q0 - window + 1, q0 + 127] are never loaded: a
 // 129-wide window touches at most two 128-key tiles per query tile.
@@ -57,7 +61,6 @@ constexpr int kPfOffK = 2 * kPfQBytes;                 // 2 stages
 constexpr int kPfOffV = kPfOffK + 2 * kPfKBytes;       // 196608
 constexpr int kPfOffBar = kPfOffV + kPfVBytes;         // 229376
 constexpr int kPfSmemBytes = kPfOffBar + 256 + 1024;   // barriers + alignment slack
-constexpr float kRescaleLog2 = 8.0f;
 
 struct PrefillParams {
   const int32_t* cu_seqlens;  // [num_seqs + 1]
@@ -347,72 +350,88 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_load128_sync(tS, s);
         const bool full_tile = (kpos0 + kPfTile - 1 <= it.q0) &&
                                (p.window == 0 || (it.q0 + kPfTile - 1) - kpos0 <= p.window - 1);
-        // Row max of the raw scores (the scale is positive, so it commutes with
-        // max), as 8 independent chains to keep the dependency depth short.
-        float mx8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-        if (full_tile) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmax3(mx8[c & 7], s[2 * c], s[2 * c + 1]);
-        } else {
+        if (!full_tile) {
           const int hi_k = qpos - kpos0;                                  // keys <= hi_k visible
           const int lo_k = p.window > 0 ? qpos - p.window + 1 - kpos0 : -1;  // keys >= lo_k visible
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            s[c] = (c <= hi_k && c >= lo_k) ? s[c] : -INFINITY;
-            mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-          }
+          for (int c = 0; c < 128; ++c) s[c] = (c <= hi_k && c >= lo_k) ? s[c] : -INFINITY;
         }
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7]));
-        const float m_new = fmaxf(m, mx * p.scale_log2);
-        float alpha = 1.f;
-        bool rescale_o = false;
-        if (m_new - m > kRescaleLog2) {  // false when both are -inf (NaN compare)
-          alpha = ex2(m - m_new);
-          l *= alpha;
-          lr *= alpha;
-          m = m_new;
-          rescale_o = (t > 0);
-        }
-        const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        // P = 2^(s*scale - m), rounded to bf16 for the PV product.  Two row sums:
-        // the unrounded values (lse, exact to fp32) and the rounded ones, which
-        // normalise the output, so that out = sum_j P~_j v_j / (sum_j P~_j + sink)
-        // weights the value rows by exactly the P that multiplied them.
-        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-        const float2 nm2 = make_float2(neg_m, neg_m);
-        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 acr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // Moves the reference m up to the row max of this tile where need is
+        // set (rescaling l, lr and, on later tiles, O by 2^(m_old - m_new)).
+        // The whole warp takes part: the O rescale is a warp-wide TMEM access.
+        auto move_max = [&](bool need) {
+          float mx8[8];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+          for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float2 x = fma2(make_float2(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]), sc2, nm2);
-            const float2 e = make_float2(ex2(x.x), ex2(x.y));
-            pk[c] = pack_bf16(e.x, e.y);
-            acc[c & 1] = add2(acc[c & 1], e);
-            add_bf16x2(acr[c & 1], pk[c]);
+          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmax3(mx8[c & 7], s[2 * c], s[2 * c + 1]);
+          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                                 fmaxf(mx8[6], mx8[7]));
+          const float m_new = fmaxf(m, mx * p.scale_log2);
+          float alpha = 1.f;
+          bool rescale_o = false;
+          if (need && m_new > m) {
+            alpha = ex2(m - m_new);  // 0 when m was -inf
+            l *= alpha;
+            lr *= alpha;
+            m = m_new;
+            rescale_o = (t > 0);
           }
-          tmem_st32(tS + 32 * half, pk);
+          // O of the previous tile is complete here: S_i(t) was committed after PV_i(t-1).
+          if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_load32_sync(tO + c * 32, o);
+              const float a_ = rescale_o ? alpha : 1.f;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a_);
+              tmem_st32(tO + c * 32, o);
+            }
+          }
+        };
+        // P = 2^(s*scale - m), rounded to bf16 for the PV product, written over
+        // the first 64 columns of S.  Two row sums: the unrounded values (lse,
+        // exact to fp32) and the rounded ones, which normalise the output, so
+        // that out = sum_j P~_j v_j / (sum_j P~_j + sink) weights the value rows
+        // by exactly the P that multiplied them.
+        float2 a, ar;
+        auto exps = [&]() {
+          const float neg_m = (m == -INFINITY) ? 0.f : -m;
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 nm2 = make_float2(neg_m, neg_m);
+          float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          float2 acr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float2 x = fma2(make_float2(s[64 * half + 2 * c], s[64 * half + 2 * c + 1]), sc2, nm2);
+              const float2 e = make_float2(ex2(x.x), ex2(x.y));
+              pk[c] = pack_bf16(e.x, e.y);
+              acc[c & 1] = add2(acc[c & 1], e);
+              add_bf16x2(acr[c & 1], pk[c]);
+            }
+            tmem_st32(tS + 32 * half, pk);
+          }
+          a = add2(acc[0], acc[1]);
+          ar = add2(acr[0], acr[1]);
+        };
+        // The reference m is the sink's logit (or, with no sink, the first row
+        // max), moved only when this tile's P would leave the safe range: P is
+        // scale-free in bf16 and fp32, so the only hazards are overflow (a sum
+        // above 2^64) and a row with no reference yet.
+        if (__any_sync(0xffffffffu, m == -INFINITY)) move_max(m == -INFINITY);
+        exps();
+        const auto unsafe = [&]() { return !(a.x + a.y <= 0x1p64f); };  // also NaN
+        if (__any_sync(0xffffffffu, unsafe())) {
+          move_max(unsafe());
+          tmem_wait_st();  // the first P stores are complete before they are overwritten
+          exps();
         }
-        const float2 a = add2(acc[0], acc[1]), ar = add2(acr[0], acr[1]);
         l += a.x + a.y;
         lr += ar.x + ar.y;
-        // O of the previous tile is complete here: S_i(t) was committed after PV_i(t-1).
-        if (__any_sync(0xffffffffu, rescale_o)) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_load32_sync(tO + c * 32, o);
-            const float a_ = rescale_o ? alpha : 1.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a_);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[i]);

@@ -134,9 +134,23 @@ def test_rescale_path_with_growing_scores():
     x.k = (x.k.float() * 0.25 + ramp * x.q[:, :1].float().sign()).to(torch.bfloat16)
     out, lse = run_gpu(x, 0, torch.float32)
     ro, rl = oracle.prefill(x.q, x.k, x.v, None, 0, x.cu_seqlens)
-    # Attention here is nearly one-hot (|out| ~ |v|) and P runs up to 2^8
-    # against stale running maxima; the flat bound holds for fp32 output.
+    # Attention here is nearly one-hot (|out| ~ |v|); the scaled scores grow
+    # by ~96 (base 2) along the keys, so later tiles overflow the first tile's
+    # reference and move it (O rescaled); the flat bound holds for fp32 output.
     P.check(out, ro, lse, rl, what="rescale")
+
+
+@pytest.mark.parametrize("window", [0, 300])
+def test_reference_moves_above_the_sink(window):
+    """Scores far above the sink logit (base-2 spread ~23 per key): P against
+    the sink's reference overflows and the kernel moves it, on the first tile
+    of a row and on later ones."""
+    x = W.prefill_inputs([1000, 300], hq=8, hkv=2, seed=9)
+    x.q = (x.q.float() * 4).to(torch.bfloat16)
+    x.k = (x.k.float() * 4).to(torch.bfloat16)
+    out, lse = run_gpu(x, window, torch.float32)
+    ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+    P.check(out, ro, lse, rl, what=f"reference moves W={window}")
 
 
 # ----------------------------------------------------------------------------
