@@ -85,13 +85,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // complete within kWaitTimeoutNs, or if another role already raised *abort.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
                                              volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  // The clock is read only every 256 failed polls (it starts at the first
+  // such read), so a hand-off that completes within a few polls costs no
+  // timer reads; the bound is kWaitTimeoutNs after 256 polls.
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & 255u) == 255u) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitTimeoutNs) {
         record_status(5 /* MIMO_ERR_TIMEOUT */);
         *abort = 1;
         return false;
