@@ -32,15 +32,21 @@ constexpr int kDecKBytes = kDecTileKeys * 192 * 2;   // 24576
 constexpr int kDecVBytes = kDecTileKeys * 128 * 2;   // 16384
 constexpr int kDecStageBytes = kDecKBytes + kDecVBytes;
 constexpr int kDecThreads = 160;                     // 4 consumer warps + 1 producer warp
+constexpr int kDecQRow = 400;                        // Q tile row stride (384 B + 16: ldmatrix rows on distinct banks)
+constexpr int kDecQBytes = 16 * kDecQRow;
 constexpr int dec_smem_bytes(int stages, int tile_rows = kDecTileKeys) {
-  return stages * 5 * tile_rows * 128 + 1024 /*align*/ + 128 /*barriers*/;
+  return stages * 5 * tile_rows * 128 + 128 /*barriers*/ + kDecQBytes + 1024 /*align*/;
 }
+// The end-of-split merge reuses the stage ring: [4 warps][16 rows][kDecORow]
+// partial O (rows padded so that neither the fragment writes nor the row
+// reads pile onto a few banks), then 3 x [4][16] floats (max, sum, rounded sum).
+constexpr int kDecORow = 136;
+constexpr int kDecMergeBytes = 4 * 16 * kDecORow * 4 + 3 * 4 * 16 * 4;
 constexpr int kDecRingStages = 3;                    // small rings: the whole ring in flight
 constexpr int kDecRingRows = 48;                     // rows of a ring tile (3 x 48 >= 129 slots)
-static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kDecRingStages * 5 * kDecRingRows * 128, "merge buffer fits");
+static_assert(kDecMergeBytes <= kDecRingStages * 5 * kDecRingRows * 128, "merge buffer fits");
 constexpr int kDecSmemBytes = dec_smem_bytes(kDecStages);
-// the end-of-split merge reuses the stage ring: [4 warps][16 rows][128] + 3 x [4][16] floats
-static_assert(4 * 16 * 128 * 4 + 3 * 4 * 16 * 4 <= kDecShortStages * kDecStageBytes, "merge buffer fits");
+static_assert(kDecMergeBytes <= kDecShortStages * kDecStageBytes, "merge buffer fits");
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // [B, Hq, 192]
@@ -102,7 +108,9 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   constexpr int kStageBytes = 5 * kBox;          // K: 3 boxes, V: 2 boxes
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
   uint64_t* empty = full + kStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  uint64_t* q_full = empty + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(q_full + 1);
+  uint8_t* sq = smem + kStages * kStageBytes + 128;  // [16 rows][kDecQRow] Q tile
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -114,18 +122,33 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   if (p.nsplit > 1 && s0 >= s1) return;  // empty split: the combine skips it
   const int nkeys = max(0, s1 - s0);
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 128) {  // the producer lane
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 4);
     }
+    mbar_init(q_full, 1);
+    fence_mbar_init();
+    // The G query rows of this KV head: one bulk copy per 384-byte row, into
+    // rows kDecQRow apart (rows >= G are never read into a fragment).
+    mbar_arrive_expect_tx(q_full, p.G * 384);
+    const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)g * p.G) * 192;
+    for (int r = 0; r < p.G; ++r) bulk_load(sq + r * kDecQRow, qg + r * 192, 384, q_full);
+  }
+  if (threadIdx.x == 0) {
     // sampled once, so every thread of the CTA sees the same decision
     *abort_flag = timed_out_before() ? 1 : 0;
-    fence_mbar_init();
   }
   __syncthreads();
-  // after a recorded timeout elsewhere, return at entry: nothing is read or written
-  if (*abort_flag) return;
+  // after a recorded timeout elsewhere, return at entry: nothing is written
+  // (the Q rows requested above land before the CTA leaves)
+  if (*abort_flag) {
+    if (threadIdx.x == 128) {
+      volatile int keep_waiting = 0;
+      wait_bounded(q_full, 0, &keep_waiting);
+    }
+    return;
+  }
   const int tile = p.tile;
   // tiles streamed: those holding the unit's keys, or every tile of a small ring
   const int ntiles = p.spec_tiles > 0 ? p.spec_tiles : (nkeys + tile - 1) / tile;
@@ -155,20 +178,18 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     // ------------------------------------------------------------ consumers
     const int r0 = lane >> 2;        // rows (heads) r0 and r0 + 8
     const int cq = (lane & 3) * 2;   // column pair within an 8-wide block
-    // Q fragments for all 12 k-steps of 16 dims; rows >= G are zero.
+    // Q fragments for all 12 k-steps of 16 dims (ldmatrix.x4: lanes 0-15 give
+    // rows 0-15 at dims +0, lanes 16-31 the same rows at dims +8); rows >= G are zero.
     uint32_t qa[12][4];
     {
-      const int h0 = g * p.G + r0, h1 = g * p.G + r0 + 8;
       const bool v0 = r0 < p.G, v1 = r0 + 8 < p.G;
-      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (v0 ? h0 : 0)) * 192);
-      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (v1 ? h1 : 0)) * 192);
+      if (!wait_bounded(q_full, 0, abort_flag)) return;
+      const uint32_t qrow = smem_u32(sq) + (lane & 15) * kDecQRow + (lane >> 4) * 16;
 #pragma unroll
       for (int kk = 0; kk < 12; ++kk) {
-        const int d = kk * 16 + cq;
-        qa[kk][0] = v0 ? __ldg(q0 + d / 2) : 0u;
-        qa[kk][1] = v1 ? __ldg(q1 + d / 2) : 0u;
-        qa[kk][2] = v0 ? __ldg(q0 + (d + 8) / 2) : 0u;
-        qa[kk][3] = v1 ? __ldg(q1 + (d + 8) / 2) : 0u;
+        ldsm_x4(qrow + kk * 32, qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+        if (!v0) qa[kk][0] = qa[kk][2] = 0u;
+        if (!v1) qa[kk][1] = qa[kk][3] = 0u;
       }
     }
     float o[16][4];
@@ -286,17 +307,15 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     lr1 += __shfl_xor_sync(0xffffffffu, lr1, 1);
     lr1 += __shfl_xor_sync(0xffffffffu, lr1, 2);
     asm volatile("bar.sync 1, 128;" ::: "memory");  // all consumers done with the stages
-    float* so = reinterpret_cast<float*>(smem);      // [4 warps][16 rows][128]
-    float* sm = so + 4 * 16 * 128;                   // [4][16] max
+    float* so = reinterpret_cast<float*>(smem);      // [4 warps][16 rows][kDecORow]
+    float* sm = so + 4 * 16 * kDecORow;              // [4][16] max
     float* sl = sm + 4 * 16;                         // [4][16] sum
     float* slr = sl + 4 * 16;                        // [4][16] sum of the rounded P
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       const int col = n * 8 + cq;
-      so[(warp * 16 + r0) * 128 + col] = o[n][0];
-      so[(warp * 16 + r0) * 128 + col + 1] = o[n][1];
-      so[(warp * 16 + r0 + 8) * 128 + col] = o[n][2];
-      so[(warp * 16 + r0 + 8) * 128 + col + 1] = o[n][3];
+      *reinterpret_cast<float2*>(so + (warp * 16 + r0) * kDecORow + col) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(so + (warp * 16 + r0 + 8) * kDecORow + col) = make_float2(o[n][2], o[n][3]);
     }
     if ((lane & 3) == 0) {
       sm[warp * 16 + r0] = m0;
@@ -307,10 +326,11 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       slr[warp * 16 + r0 + 8] = lr1;
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    // 128 threads: thread -> (row = tid / 8, 16 columns)
+    // 128 threads: thread -> (row = tid / 8; columns 4 (tid & 7) + 32 j, j = 0..3,
+    // so that the 8 threads of a row read 128 contiguous bytes per access)
     const int tid = threadIdx.x;
     const int row = tid >> 3;
-    const int c0 = (tid & 7) * 16;
+    const int cb = (tid & 7) * 4;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w * 16 + row]);
@@ -322,13 +342,19 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       Ls += wgt[w] * sl[w * 16 + row];
       Lrs += wgt[w] * slr[w * 16 + row];
     }
-    float acc[16];
+    float4 acc[4];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float a = 0.f;
+    for (int j = 0; j < 4; ++j) {
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int w = 0; w < 4; ++w) a += wgt[w] * so[(w * 16 + row) * 128 + c0 + e];
-      acc[e] = a;
+      for (int w = 0; w < 4; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(so + (w * 16 + row) * kDecORow + cb + 32 * j);
+        a.x += wgt[w] * v.x;
+        a.y += wgt[w] * v.y;
+        a.z += wgt[w] * v.z;
+        a.w += wgt[w] * v.w;
+      }
+      acc[j] = a;
     }
     if (row < p.G) {
       const int h = g * p.G + row;
@@ -344,32 +370,24 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
           Lrf = Lrs * scl + ps;
         }
         const float f = (Lrf > 0.f) ? p.v_scale * scl / Lrf : 0.f;
-        const size_t ob = ((size_t)b * p.Hq + h) * 128 + c0;
-        if (p.out_f32) {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob);
+        const size_t ob = ((size_t)b * p.Hq + h) * 128 + cb;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_float4(acc[4 * e] * f, acc[4 * e + 1] * f, acc[4 * e + 2] * f, acc[4 * e + 3] * f);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob);
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            uint4 u;
-            u.x = pack_bf16(acc[8 * e + 0] * f, acc[8 * e + 1] * f);
-            u.y = pack_bf16(acc[8 * e + 2] * f, acc[8 * e + 3] * f);
-            u.z = pack_bf16(acc[8 * e + 4] * f, acc[8 * e + 5] * f);
-            u.w = pack_bf16(acc[8 * e + 6] * f, acc[8 * e + 7] * f);
-            dst[e] = u;
+        for (int j = 0; j < 4; ++j) {
+          if (p.out_f32) {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + ob + 32 * j) =
+                make_float4(acc[j].x * f, acc[j].y * f, acc[j].z * f, acc[j].w * f);
+          } else {
+            *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + ob + 32 * j) =
+                make_uint2(pack_bf16(acc[j].x * f, acc[j].y * f), pack_bf16(acc[j].z * f, acc[j].w * f));
           }
         }
         if (p.lse && (tid & 7) == 0)
           p.lse[(size_t)b * p.Hq + h] = (Lf > 0.f) ? (Mf * 0.6931471805599453f + logf(Lf)) : -INFINITY;
       } else {
         const size_t unit = ((size_t)b * p.Hkv + g) * p.nsplit + split;
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + (unit * 16 + row) * 128 + c0);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<float4*>(p.ws_o + (unit * 16 + row) * 128 + cb + 32 * j) = acc[j];
         if ((tid & 7) == 0) {
           p.ws_ml[(unit * 16 + row) * 4 + 0] = M;
           p.ws_ml[(unit * 16 + row) * 4 + 1] = Ls;
