@@ -90,7 +90,11 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr) {
 }
 
 // One work item, decoded.  Items are numbered heaviest query tile first;
-// within a query tile, key/value head pair then sequence.
+// within a query tile, sequence then key/value head pair, so that a
+// sequence's items sit together: in a pack of mixed lengths, where the long
+// sequences alone have the high query tiles, this spreads the work evenly
+// over the CTAs' round-robin shares (busiest CTA 1.04x the mean for 16
+// sequences of 512..8192 tokens, against 1.41x with the sequence innermost).
 struct PfItem {
   int b0, len, q0, g, h0, j_lo, n_kt;
   bool has1, valid;
@@ -104,9 +108,10 @@ __device__ __forceinline__ PfItem pf_decode(const PrefillParams& p, int item) {
   PfItem it;
   const int per_q = p.Hkv * p.pairs_per_group * p.num_seqs;
   const int qt = p.num_qtiles - 1 - item / per_q;
-  int rem = item % per_q;
-  const int seq = rem % p.num_seqs;
-  const int pair = rem / p.num_seqs;
+  const int rem = item % per_q;
+  const int npairs = p.Hkv * p.pairs_per_group;
+  const int seq = rem / npairs;
+  const int pair = rem % npairs;
   it.g = pair / p.pairs_per_group;
   const int pp = pair % p.pairs_per_group;
   it.h0 = it.g * p.G + 2 * pp;
