@@ -231,7 +231,7 @@ def test_output_only_16_byte_aligned(odt):
 
 # ----------------------------------------------------------------------------
 # sliding window with the key/value group packed into the MMA rows
-# (G = Hq/Hkv in {8, 16, 32}; N = roundup16(W + 128/G - 1) <= 160, else the
+# (G = Hq/Hkv in {8, 16, 32}; N = roundup16(W + 256/G - 1) <= 160, else the
 # per-head kernel takes the call: the largest packed windows are 129 at G=8,
 # 145 at G=16 and 153 at G=32, and the next window up crosses to the other kernel)
 
