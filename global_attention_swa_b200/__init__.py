@@ -22,7 +22,10 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmimo_attn.so")
+#: MIMO_ATTN_CHECKED=1 in the environment loads the bounds-checked build
+#: (libmimo_attn_checked.so: every kernel checks its row indices, see the header)
+CHECKED = os.environ.get("MIMO_ATTN_CHECKED", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libmimo_attn_checked.so" if CHECKED else "libmimo_attn.so")
 
 MIMO_OK = 0
 MIMO_ERR_INVALID_ARG = 1
@@ -30,6 +33,7 @@ MIMO_ERR_UNSUPPORTED = 2
 MIMO_ERR_CUDA = 3
 MIMO_ERR_WORKSPACE = 4
 MIMO_ERR_TIMEOUT = 5
+MIMO_ERR_BOUNDS = 6
 MIMO_DTYPE_BF16 = 0
 MIMO_DTYPE_F32 = 1
 
@@ -48,6 +52,9 @@ EXPORTED = (
     "mimo_attn_decode_merge",
     "mimo_attn_prefill_backward_workspace_size",
     "mimo_attn_prefill_backward",
+    "mimo_attn_is_checked_build",
+    "mimo_attn_checked_site",
+    "mimo_attn_checked_selftest",
 )
 
 
@@ -72,7 +79,8 @@ class Dims(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing; build it with global_attention_swa_b200._build.build()")
+            f"{LIB_PATH} is missing; build it with global_attention_swa_b200._build.build("
+            f"{'checked=True' if CHECKED else ''})")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     dp = ctypes.POINTER(Dims)
@@ -103,6 +111,12 @@ def _load():
     lib.mimo_attn_prefill_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
                                                vp, vp, vp, vp, vp, sz, vp]
     lib.mimo_attn_prefill_backward.restype = i32
+    lib.mimo_attn_is_checked_build.argtypes = []
+    lib.mimo_attn_is_checked_build.restype = i32
+    lib.mimo_attn_checked_site.argtypes = [vp]
+    lib.mimo_attn_checked_site.restype = i32
+    lib.mimo_attn_checked_selftest.argtypes = [vp]
+    lib.mimo_attn_checked_selftest.restype = i32
     return lib
 
 
@@ -409,6 +423,29 @@ def mimo_attn_set_device_status(code, stream=None, device=None):
         stream.device if stream is not None else _current_device())
     with _on_device(dev):
         _check(lib.mimo_attn_set_device_status(int(code), _stream(stream, dev)))
+
+
+def mimo_attn_is_checked_build():
+    """True when the loaded library is the bounds-checked build."""
+    return bool(lib.mimo_attn_is_checked_build())
+
+
+def mimo_attn_checked_site(stream=None, device=None):
+    """Synchronise the stream; return (and clear) the first site at which the
+    checked build caught a row index outside its buffer, 0 if none."""
+    dev = torch.device(device) if device is not None else (
+        stream.device if stream is not None else _current_device())
+    with _on_device(dev):
+        return int(lib.mimo_attn_checked_site(_stream(stream, dev)))
+
+
+def mimo_attn_checked_selftest(stream=None, device=None):
+    """Checked build only: launch the one-thread kernel whose row check fails
+    without touching memory (see include/mimo_attn.h)."""
+    dev = torch.device(device) if device is not None else (
+        stream.device if stream is not None else _current_device())
+    with _on_device(dev):
+        _check(lib.mimo_attn_checked_selftest(_stream(stream, dev)))
 
 
 def default_scale(dqk=192):

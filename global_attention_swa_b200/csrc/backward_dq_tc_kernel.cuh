@@ -35,6 +35,9 @@
 
 #include "backward_kernel.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 9  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kBdThreads = 192;
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(kBdThreads, 1)
     const int r = threadIdx.x;  // TMEM lane == query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const int q = q0 + r;
-    const bool live = q < len;
+    const bool live = q < len && MIMO_ROW_OK((long long)(b0 + q) * p.Hq + h, (long long)p.total * p.Hq);
     const size_t li = (size_t)h * p.total + b0 + q;
     const float lse2 = live ? p.lse[li] * 1.4426950408889634f : 0.f;
     const float Dq = live ? p.D[li] : 0.f;

@@ -27,6 +27,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 7  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kBwTile = 64;
@@ -327,14 +330,17 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_dq_kernel(const BackwardPar
 
   // write dq * scale for valid rows
   const int ra = r0 + gr, rb = ra + 8;
+  const long long dq_rows = (long long)p.total * p.Hq;
+  const bool oka = ra < qv && MIMO_ROW_OK((long long)(b0 + q0 + ra) * p.Hq + h, dq_rows);
+  const bool okb = rb < qv && MIMO_ROW_OK((long long)(b0 + q0 + rb) * p.Hq + h, dq_rows);
 #pragma unroll
   for (int n = 0; n < 24; ++n) {
     const int col = 8 * n + 2 * t4;
-    if (ra < qv) {
+    if (oka) {
       float* dst = p.dq + ((size_t)(b0 + q0 + ra) * p.Hq + h) * kBwQK + col;
       *reinterpret_cast<float2*>(dst) = make_float2(dq[n][0] * p.scale, dq[n][1] * p.scale);
     }
-    if (rb < qv) {
+    if (okb) {
       float* dst = p.dq + ((size_t)(b0 + q0 + rb) * p.Hq + h) * kBwQK + col;
       *reinterpret_cast<float2*>(dst) = make_float2(dq[n][2] * p.scale, dq[n][3] * p.scale);
     }
@@ -518,13 +524,16 @@ __global__ void __launch_bounds__(kBkThreads, 1) bwd_dkv_kernel(const BackwardPa
   constexpr int D = kDV ? kBwV : kBwQK;
   float* out = kDV ? p.dv : p.dk;
   const int ra = kw + gr, rb = ra + 8;
+  const long long kv_rows = (long long)p.total * p.Hkv;
+  const bool oka = ra < kv && MIMO_ROW_OK((long long)(b0 + k0 + ra) * p.Hkv + g, kv_rows);
+  const bool okb = rb < kv && MIMO_ROW_OK((long long)(b0 + k0 + rb) * p.Hkv + g, kv_rows);
 #pragma unroll
   for (int n = 0; n < NB; ++n) {
     const int col = 8 * n + 2 * t4;
-    if (ra < kv)
+    if (oka)
       *reinterpret_cast<float2*>(out + ((size_t)(b0 + k0 + ra) * p.Hkv + g) * D + col) =
           make_float2(acc[n][0] * f, acc[n][1] * f);
-    if (rb < kv)
+    if (okb)
       *reinterpret_cast<float2*>(out + ((size_t)(b0 + k0 + rb) * p.Hkv + g) * D + col) =
           make_float2(acc[n][2] * f, acc[n][3] * f);
   }

@@ -37,6 +37,9 @@
 
 #include "backward_kernel.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 8  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kBtThreads = 192;
@@ -263,6 +266,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       const int qp = (qt_lo + j % nq) * kBtQ + (r & (kBtQ - 1));
       if (qp >= len) return 0.f;
       const size_t gi = (size_t)(g * p.G + j / nq) * p.total + b0 + qp;
+      if (!MIMO_ROW_OK(gi, (long long)p.Hq * p.total)) return 0.f;
       return r < kBtQ ? p.lse[gi] * 1.4426950408889634f : p.D[gi];
     };
     bool ok = items > 0;
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
     // ---------------- epilogue: dV * v_scale and dK * scale for valid keys
     if (ok && wait_bounded(done, 0, abort_flag)) {
       tc_fence_after();
-      const bool valid = r < kv;
+      const bool valid = r < kv && MIMO_ROW_OK((long long)(b0 + key) * p.Hkv + g, (long long)p.total * p.Hkv);
       float* dvr = p.dv + ((size_t)(b0 + key) * p.Hkv + g) * kBwV;
       float* dkr = p.dk + ((size_t)(b0 + key) * p.Hkv + g) * kBwQK;
 #pragma unroll 1

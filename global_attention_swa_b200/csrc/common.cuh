@@ -29,6 +29,27 @@ __device__ __forceinline__ bool timed_out_before() {
   return *reinterpret_cast<volatile int*>(&g_device_status) == 5 /* MIMO_ERR_TIMEOUT */;
 }
 
+// ---------------------------------------------------------------- checked build
+// Built with -DMIMO_CHECKED (libmimo_attn_checked.so), every kernel checks the
+// row index it forms for a global read or write against the row count of that
+// buffer before the access.  A miss records MIMO_ERR_BOUNDS in the device
+// status word and the site (MIMO_FILE_ID * 10000 + line) in g_checked_site,
+// and the access is skipped.  In the normal build the check is the constant
+// true and costs nothing.  Each kernel header defines MIMO_FILE_ID.
+__device__ int g_checked_site;
+#ifdef MIMO_CHECKED
+__device__ __forceinline__ bool checked_row(long long i, long long n, int site) {
+  if (i >= 0 && i < n) return true;
+  atomicCAS(&g_device_status, 0, 6 /* MIMO_ERR_BOUNDS */);
+  atomicCAS(&g_checked_site, 0, site);
+  return false;
+}
+#define MIMO_ROW_OK(i, n) \
+  (::mimo::checked_row(static_cast<long long>(i), static_cast<long long>(n), MIMO_FILE_ID * 10000 + __LINE__))
+#else
+#define MIMO_ROW_OK(i, n) ((void)sizeof(i), (void)sizeof(n), true)  // unevaluated
+#endif
+
 // A packed sequence [b0, b0 + len) fits the call: it starts inside the token
 // range, its length is non-negative and at most max_seqlen, and it ends by
 // `total`.  The prefill and backward kernels check every sequence they touch

@@ -25,6 +25,9 @@
 
 #include "decode_kernel.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 4  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kD8TileKeys = 64;
@@ -107,7 +110,8 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
     uint32_t qa[12][4];
     {
       const int h0 = g * p.G + r0, h1 = g * p.G + r0 + 8;
-      const bool v0 = r0 < p.G, v1 = r0 + 8 < p.G;
+      const bool v0 = r0 < p.G && MIMO_ROW_OK((long long)b * p.Hq + h0, (long long)p.B * p.Hq);
+      const bool v1 = r0 + 8 < p.G && MIMO_ROW_OK((long long)b * p.Hq + h1, (long long)p.B * p.Hq);
       const uint2* q0 = reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.Hq + (v0 ? h0 : 0)) * 192);
       const uint2* q1 = reinterpret_cast<const uint2*>(p.q + ((size_t)b * p.Hq + (v1 ? h1 : 0)) * 192);
 #pragma unroll
@@ -296,7 +300,9 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
       for (int w = 0; w < 4; ++w) a += wgt[w] * so[(w * 16 + row) * 128 + c0 + e];
       acc[e] = a;
     }
-    if (row < p.G) {
+    if (row < p.G &&
+        (p.nsplit == 1 ? MIMO_ROW_OK((long long)b * p.Hq + g * p.G + row, (long long)p.B * p.Hq)
+                       : MIMO_ROW_OK(((long long)b * p.Hkv + g) * p.nsplit + split, (long long)p.B * p.Hkv * p.nsplit))) {
       const int h = g * p.G + row;
       if (p.nsplit == 1) {
         const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;

@@ -22,6 +22,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 3  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kDecTileKeys = 64;
@@ -131,9 +134,11 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
     fence_mbar_init();
     // The G query rows of this KV head: one bulk copy per 384-byte row, into
     // rows kDecQRow apart (rows >= G are never read into a fragment).
-    mbar_arrive_expect_tx(q_full, p.G * 384);
+    const bool q_ok = MIMO_ROW_OK((long long)b * p.Hq + (long long)(g + 1) * p.G - 1, (long long)p.B * p.Hq);
+    mbar_arrive_expect_tx(q_full, q_ok ? p.G * 384 : 0);
     const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)g * p.G) * 192;
-    for (int r = 0; r < p.G; ++r) bulk_load(sq + r * kDecQRow, qg + r * 192, 384, q_full);
+    if (q_ok)
+      for (int r = 0; r < p.G; ++r) bulk_load(sq + r * kDecQRow, qg + r * 192, 384, q_full);
   }
   if (threadIdx.x == 0) {
     // sampled once, so every thread of the CTA sees the same decision
@@ -356,7 +361,9 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       }
       acc[j] = a;
     }
-    if (row < p.G) {
+    if (row < p.G &&
+        (p.nsplit == 1 ? MIMO_ROW_OK((long long)b * p.Hq + g * p.G + row, (long long)p.B * p.Hq)
+                       : MIMO_ROW_OK(((long long)b * p.Hkv + g) * p.nsplit + split, (long long)p.B * p.Hkv * p.nsplit))) {
       const int h = g * p.G + row;
       if (p.nsplit == 1) {
         // fold the sink: it joins the normaliser only
@@ -413,8 +420,10 @@ __global__ void __launch_bounds__(256)
   const int g = h / p.G, row = h % p.G;
   int lo, hi;
   decode_range(p, p.seqlens[b], lo, hi);
-  const int nused = min(p.nsplit, max(0, (hi - lo + p.chunk - 1) / p.chunk));
+  int nused = min(p.nsplit, max(0, (hi - lo + p.chunk - 1) / p.chunk));
   const size_t unit0 = ((size_t)b * p.Hkv + g) * p.nsplit;
+  if (nused > 0 && !MIMO_ROW_OK(unit0 + nused - 1, (long long)p.B * p.Hkv * p.nsplit)) nused = 0;
+  if (!MIMO_ROW_OK((long long)b * p.Hq + h, (long long)p.B * p.Hq)) return;
   const float sg = p.sinks ? p.sinks[h] * 1.4426950408889634f : -INFINITY;
   float M = sg;
   for (int c = 0; c < nused; ++c) M = fmaxf(M, p.ws_ml[((unit0 + c) * 16 + row) * 4]);

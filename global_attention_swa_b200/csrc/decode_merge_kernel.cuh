@@ -13,6 +13,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 5  // site numbers of the checked build
+
 namespace mimo {
 
 struct DecodeMergeParams {
@@ -33,6 +36,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecodeMergePara
   const int b = wid / p.Hq, h = wid % p.Hq;
   const size_t bh = (size_t)b * p.Hq + h;
   const size_t stride = (size_t)p.B * p.Hq;  // between parts
+  if (!MIMO_ROW_OK(bh + (size_t)(p.R - 1) * stride, (long long)p.R * stride)) return;
   const float sg = p.sinks ? p.sinks[h] : -INFINITY;
   float M = sg;
   for (int r = 0; r < p.R; ++r) M = fmaxf(M, p.part_lse[r * stride + bh]);

@@ -23,6 +23,19 @@
 #include "prefill_kernel.cuh"
 #include "prefill_swa_kernel.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 10  // site numbers of the checked build
+
+#ifdef MIMO_CHECKED
+namespace mimo {
+// One row index past a 4-row buffer, checked and not used for any access.
+__global__ void checked_selftest_kernel() {
+  const volatile int row = 4;
+  if (MIMO_ROW_OK(row, 4)) record_status(3 /* not reached: the check fails */);
+}
+}  // namespace mimo
+#endif
+
 namespace {
 
 thread_local std::string g_last_error;
@@ -754,6 +767,35 @@ mimo_status_t mimo_attn_device_status(void* stream) {
     return st;
   if (v == 0) return ok();
   return fail(static_cast<mimo_status_t>(v), "device status %d recorded by a kernel", v);
+}
+
+int mimo_attn_is_checked_build(void) {
+#ifdef MIMO_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int mimo_attn_checked_site(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return 0;
+  int v = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&v, mimo::g_checked_site, sizeof(int)) != cudaSuccess) return 0;
+  if (cudaMemcpyToSymbol(mimo::g_checked_site, &zero, sizeof(int)) != cudaSuccess) return 0;
+  return v;
+}
+
+mimo_status_t mimo_attn_checked_selftest(void* stream) {
+#ifdef MIMO_CHECKED
+  mimo::checked_selftest_kernel<<<1, 1, 0, (cudaStream_t)stream>>>();
+  mimo_status_t st;
+  if ((st = cuda_check(cudaGetLastError(), "checked self-test launch"))) return st;
+  return ok();
+#else
+  (void)stream;
+  return fail(MIMO_ERR_UNSUPPORTED, "not the checked build");
+#endif
 }
 
 mimo_status_t mimo_attn_set_device_status(int code, void* stream) {

@@ -48,6 +48,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 1  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kPfThreads = 384;
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_before();
       mbar_arrive(&o_empty[i]);
       ++n;
-      if (qpos < it.len) {
+      if (qpos < it.len && MIMO_ROW_OK((long long)(it.b0 + qpos) * p.Hq + h, (long long)p.total * p.Hq)) {
         const int tok = it.b0 + qpos;
         const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
         const size_t ob = ((size_t)tok * p.Hq + h) * 128;

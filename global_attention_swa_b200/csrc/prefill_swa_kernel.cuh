@@ -37,6 +37,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 2  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kSwThreads = 448;
@@ -387,9 +390,10 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tmem_load16_sync(tbase + lane_off + kSwColSum, rs);  // rounded-P row sum (16 equal columns)
       const float lr = rs[0] + mlv.z;
       const int qpos = it.q0 + blk * p.QB + a;
-      const bool live = qpos < it.len;
-      const int tok = it.b0 + qpos;
       const int hg = it.g * p.G + hh;
+      const bool live =
+          qpos < it.len && MIMO_ROW_OK((long long)(it.b0 + qpos) * p.Hq + hg, (long long)p.total * p.Hq);
+      const int tok = it.b0 + qpos;
       const float f = (lr > 0.f) ? p.v_scale / lr : 0.f;
       const size_t ob = ((size_t)tok * p.Hq + hg) * 128;
       // O in two 64-column halves (registers: 448 threads leave 128 per thread);

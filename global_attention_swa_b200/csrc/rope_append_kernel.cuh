@@ -19,6 +19,9 @@
 
 #include "common.cuh"
 
+#undef MIMO_FILE_ID
+#define MIMO_FILE_ID 6  // site numbers of the checked build
+
 namespace mimo {
 
 constexpr int kRaThreads = 192;
@@ -86,6 +89,7 @@ __global__ void __launch_bounds__(kRaThreads) rope_append_kernel(const RopeAppen
     // ---- query heads [16 grp, 16 grp + 16), in place
     const int h0 = grp * kRaHeadsPerCta;
     const int nh = min(kRaHeadsPerCta, p.Hq - h0);
+    if (!MIMO_ROW_OK((long long)b * p.Hq + h0 + nh - 1, (long long)p.B * p.Hq)) return;
     __nv_bfloat16* q = p.q + ((size_t)b * p.Hq + h0) * 192;
     for (int w = threadIdx.x; w < nh * tasks; w += blockDim.x) {
       __nv_bfloat16* row = q + (w / tasks) * 192;
@@ -102,6 +106,7 @@ __global__ void __launch_bounds__(kRaThreads) rope_append_kernel(const RopeAppen
   }
   // ---- keys (rotated) and values into the cache slot
   const int slot = p.ring ? pos % p.C : pos;
+  if (!MIMO_ROW_OK((long long)b * p.C + slot, (long long)p.B * p.C)) return;
   const __nv_bfloat16* ks = p.k_new + (size_t)b * p.Hkv * 192;
   __nv_bfloat16* kd = p.k_cache + ((size_t)b * p.C + slot) * p.Hkv * 192;
   if (vec) {

@@ -55,7 +55,8 @@ typedef enum {
   MIMO_ERR_UNSUPPORTED = 2,   /* head dims other than 192/128, group > 16 ... */
   MIMO_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
   MIMO_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than required */
-  MIMO_ERR_TIMEOUT = 5        /* a bounded in-kernel wait gave up */
+  MIMO_ERR_TIMEOUT = 5,       /* a bounded in-kernel wait gave up */
+  MIMO_ERR_BOUNDS = 6         /* checked build only: an index outside its buffer (access skipped) */
 } mimo_status_t;
 
 typedef enum { MIMO_DTYPE_BF16 = 0, MIMO_DTYPE_F32 = 1 } mimo_dtype_t;
@@ -317,7 +318,8 @@ const char* mimo_attn_last_error(void);
 /*
  * Synchronises `stream`, then reads and clears the device status word that
  * bounded in-kernel waits and device-side argument checks write.  Returns
- * MIMO_OK, MIMO_ERR_TIMEOUT, MIMO_ERR_INVALID_ARG or MIMO_ERR_CUDA.
+ * MIMO_OK, MIMO_ERR_TIMEOUT, MIMO_ERR_INVALID_ARG, MIMO_ERR_BOUNDS (checked
+ * build) or MIMO_ERR_CUDA.
  */
 mimo_status_t mimo_attn_device_status(void* stream);
 
@@ -332,6 +334,28 @@ mimo_status_t mimo_attn_device_status(void* stream);
  * code and clears it.  Codes outside 0..5 return MIMO_ERR_INVALID_ARG.
  */
 mimo_status_t mimo_attn_set_device_status(int code, void* stream);
+
+/*
+ * Bounds-checked build.  The same sources compiled with -DMIMO_CHECKED give
+ * libmimo_attn_checked.so: every kernel checks each row index it forms for a
+ * global read or write against the row count of that buffer before the
+ * access.  A miss skips the access and records MIMO_ERR_BOUNDS in the device
+ * status word and its site (file number * 10000 + source line) for
+ * mimo_attn_checked_site().  The checks only catch indexing mistakes of the
+ * library itself: the host and device argument checks above come first.  In
+ * the normal build the checks compile away.
+ *
+ * mimo_attn_is_checked_build: 1 in the checked build, 0 otherwise.
+ * mimo_attn_checked_site: synchronises `stream`, returns the first recorded
+ *   site (0 if none) and clears it; always 0 in the normal build.
+ * mimo_attn_checked_selftest: checked build only (else MIMO_ERR_UNSUPPORTED):
+ *   launches one thread that checks row 4 of a 4-row buffer and touches no
+ *   memory, so that the status word then holds MIMO_ERR_BOUNDS and the site
+ *   is set; asynchronous on `stream`.
+ */
+int mimo_attn_is_checked_build(void);
+int mimo_attn_checked_site(void* stream);
+mimo_status_t mimo_attn_checked_selftest(void* stream);
 
 #ifdef __cplusplus
 }

@@ -33,6 +33,25 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+CHECKED_LIB = os.path.join(os.path.dirname(mimo.LIB_PATH), "libmimo_attn_checked.so")
+
+
+@pytest.mark.skipif(not os.path.exists(CHECKED_LIB), reason="checked build not built")
+def test_checked_build_exports_the_same_symbols_and_says_so():
+    lib = ctypes.CDLL(CHECKED_LIB)
+    for name in sorted(declared_symbols()):
+        assert hasattr(lib, name), name
+    assert lib.mimo_attn_is_checked_build() == 1
+    assert ctypes.CDLL(os.path.join(os.path.dirname(mimo.LIB_PATH), "libmimo_attn.so")
+                       ).mimo_attn_is_checked_build() == 0
+
+
+def test_selftest_is_refused_outside_the_checked_build():
+    if mimo.CHECKED:
+        pytest.skip("the checked build is loaded")
+    assert mimo.lib.mimo_attn_checked_selftest(None) == mimo.MIMO_ERR_UNSUPPORTED
+
+
 def _dims(hq=64, hkv=4, dqk=192, dv=128):
     return mimo.make_dims(hq, hkv, dqk, dv)
 
