@@ -432,11 +432,15 @@ def mimo_attn_is_checked_build():
 
 def mimo_attn_checked_site(stream=None, device=None):
     """Synchronise the stream; return (and clear) the first site at which the
-    checked build caught a row index outside its buffer, 0 if none."""
+    checked build caught a row index outside its buffer, 0 if none; raise if a
+    CUDA call failed."""
     dev = torch.device(device) if device is not None else (
         stream.device if stream is not None else _current_device())
     with _on_device(dev):
-        return int(lib.mimo_attn_checked_site(_stream(stream, dev)))
+        site = int(lib.mimo_attn_checked_site(_stream(stream, dev)))
+    if site < 0:
+        raise MimoAttnError(MIMO_ERR_CUDA, lib.mimo_attn_last_error().decode())
+    return site
 
 
 def mimo_attn_checked_selftest(stream=None, device=None):

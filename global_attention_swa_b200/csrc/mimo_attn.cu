@@ -778,11 +778,12 @@ int mimo_attn_is_checked_build(void) {
 }
 
 int mimo_attn_checked_site(void* stream) {
-  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return 0;
   int v = 0;
   const int zero = 0;
-  if (cudaMemcpyFromSymbol(&v, mimo::g_checked_site, sizeof(int)) != cudaSuccess) return 0;
-  if (cudaMemcpyToSymbol(mimo::g_checked_site, &zero, sizeof(int)) != cudaSuccess) return 0;
+  if (cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize") ||
+      cuda_check(cudaMemcpyFromSymbol(&v, mimo::g_checked_site, sizeof(int)), "read checked site") ||
+      cuda_check(cudaMemcpyToSymbol(mimo::g_checked_site, &zero, sizeof(int)), "clear checked site"))
+    return -1;
   return v;
 }
 

@@ -347,7 +347,8 @@ mimo_status_t mimo_attn_set_device_status(int code, void* stream);
  *
  * mimo_attn_is_checked_build: 1 in the checked build, 0 otherwise.
  * mimo_attn_checked_site: synchronises `stream`, returns the first recorded
- *   site (0 if none) and clears it; always 0 in the normal build.
+ *   site (0 if none) and clears it; always 0 in the normal build; -1 if a
+ *   CUDA call failed (mimo_attn_last_error() says which).
  * mimo_attn_checked_selftest: checked build only (else MIMO_ERR_UNSUPPORTED):
  *   launches one thread that checks row 4 of a 4-row buffer and touches no
  *   memory, so that the status word then holds MIMO_ERR_BOUNDS and the site
