@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(kBdThreads, 1)
   uint64_t* done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+  uint64_t* mma_drain = bars + 14;  // teardown after a timed-out wait only
+  volatile int* never_flag = reinterpret_cast<volatile int*>(bars + 15);  // never raised
 
   const int h = blockIdx.y, seq = blockIdx.z;
   const int b0 = p.cu_seqlens[seq], len = p.cu_seqlens[seq + 1] - b0;
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(kBdThreads, 1)
   const int n_kt = last_q / kBdKeys - kt_lo + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int armed_qo = 0, armed_k = 0, armed_v = 0;  // phases the producer armed (K: tiles in order)
   if (warp == 4) {
     if (lane == 0) {
       mbar_init(qo_full, 1);
@@ -114,6 +117,8 @@ __global__ void __launch_bounds__(kBdThreads, 1)
       mbar_init(v_empty, 1);
       mbar_init(s_full, 1);
       mbar_init(s_free, 128);
+      mbar_init(mma_drain, 1);
+      *never_flag = 0;
       mbar_init(dp_full, 1);
       mbar_init(ds_full, 128);
       mbar_init(done, 1);
@@ -140,6 +145,7 @@ __global__ void __launch_bounds__(kBdThreads, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(qo_full, kBdQBytes + kBdOBytes);
+      ++armed_qo;
 #pragma unroll
       for (int c = 0; c < 3; ++c) tma_load_3d(smem + kBdOffQ + c * 16384, &tm_q, qo_full, c * 64, h, b0 + q0);
 #pragma unroll
@@ -149,11 +155,13 @@ __global__ void __launch_bounds__(kBdThreads, 1)
         const int row = b0 + (kt_lo + t) * kBdKeys;
         if (t >= 2 && !wait_bounded(&k_empty[ks], ((t >> 1) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&k_full[ks], kBdKBytes);
+        ++armed_k;
 #pragma unroll
         for (int c = 0; c < 3; ++c)
           tma_load_3d(smem + kBdOffK + ks * kBdKBytes + c * 16384, &tm_k, &k_full[ks], c * 64, g, row);
         if (t >= 1 && !wait_bounded(v_empty, (t - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(v_full, kBdVBytes);
+        ++armed_v;
 #pragma unroll
         for (int c = 0; c < 2; ++c) tma_load_3d(smem + kBdOffV + c * 16384, &tm_v, v_full, c * 64, g, row);
       }
@@ -299,6 +307,18 @@ __global__ void __launch_bounds__(kBdThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // a role gave up: the loads and MMAs still in flight land before the CTA
+    // frees its TMEM and exits
+    if (warp == 4 && lane == 0) {
+      drain_armed(qo_full, armed_qo, never_flag);
+      drain_armed(&k_full[0], (armed_k + 1) / 2, never_flag);
+      drain_armed(&k_full[1], armed_k / 2, never_flag);
+      drain_armed(v_full, armed_v, never_flag);
+    }
+    if (warp == 5 && lane == 0 && nt > 0) drain_mma(mma_drain, never_flag);  // nt > 0: MMAs may have been issued
+    __syncthreads();
+  }
   if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);

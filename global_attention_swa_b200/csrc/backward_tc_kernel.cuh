@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   uint64_t* done = bars + 15;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+  uint64_t* mma_drain = bars + 18;  // teardown after a timed-out wait only
+  volatile int* never_flag = reinterpret_cast<volatile int*>(bars + 19);  // never raised
   float* sLD = reinterpret_cast<float*>(smem + kBtOffLD);
 
   // key tiles in ascending order, KV heads fastest: the longest causal loops start first
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   const int nq = qt_hi - qt_lo + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int armed_kv = 0, armed_q = 0;  // phases the producer armed: K/V once, Q/dO per item (stage j % 3)
   if (warp == 4) {
     if (lane == 0) {
       mbar_init(kv_full, 1);
@@ -130,6 +133,8 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       }
       mbar_init(dp_full, 1);
       mbar_init(ds_full, 128);
+      mbar_init(mma_drain, 1);
+      *never_flag = 0;
       mbar_init(done, 1);
       *abort_flag = timed_out_before() ? 1 : 0;
       fence_mbar_init();
@@ -154,6 +159,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(kv_full, kBtKBytes + kBtVBytes);
+      ++armed_kv;
 #pragma unroll
       for (int c = 0; c < 3; ++c) tma_load_3d(smem + kBtOffK + c * 16384, &tm_k, kv_full, c * 64, g, b0 + k0);
 #pragma unroll
@@ -165,6 +171,7 @@ __global__ void __launch_bounds__(kBtThreads, 1)
         const int row = b0 + (qt_lo + j % nq) * kBtQ;
         uint8_t* stg = smem + kBtOffStage + st * kBtStage;
         mbar_arrive_expect_tx(&q_full[st], kBtStage);
+        ++armed_q;
 #pragma unroll
         for (int c = 0; c < 3; ++c) tma_load_3d(stg + c * 8192, &tm_q, &q_full[st], c * 64, h, row);
 #pragma unroll
@@ -362,6 +369,17 @@ __global__ void __launch_bounds__(kBtThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // a role gave up: the loads and MMAs still in flight land before the CTA
+    // frees its TMEM and exits
+    if (warp == 4 && lane == 0) {
+      drain_armed(kv_full, armed_kv, never_flag);
+      for (int s = 0; s < kBtStages; ++s)
+        drain_armed(&q_full[s], armed_q > s ? (armed_q - 1 - s) / kBtStages + 1 : 0, never_flag);
+    }
+    if (warp == 5 && lane == 0 && items > 0) drain_mma(mma_drain, never_flag);  // items > 0: MMAs may have been issued
+    __syncthreads();
+  }
   if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);

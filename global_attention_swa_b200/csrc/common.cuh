@@ -243,6 +243,21 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Teardown after a role gave up (a timed-out wait anywhere in the CTA): the
+// CTA must not exit while its asynchronous copies or MMAs still write its
+// shared memory or TMEM.  drain_armed waits for the last of the `armed`
+// phases a producer armed on `bar` (each completes only when its bytes have
+// landed: nothing else arrives on it); drain_mma commits the calling thread's
+// MMAs to a fresh barrier and waits for them.  Both waits are bounded too;
+// `never` is a flag nothing raises, so only the time bound ends them.
+__device__ __forceinline__ void drain_armed(uint64_t* bar, int armed, volatile int* never) {
+  if (armed > 0) wait_bounded(bar, static_cast<uint32_t>(armed - 1) & 1u, never);
+}
+__device__ __forceinline__ void drain_mma(uint64_t* bar, volatile int* never) {
+  umma_commit(bar);
+  wait_bounded(bar, 0, never);
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

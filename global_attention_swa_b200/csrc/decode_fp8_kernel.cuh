@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kD8Stages * kD8StageBytes);
   uint64_t* empty = full + kD8Stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kD8Stages);
+  volatile int* never_flag = abort_flag + 1;  // never raised: bounds the drains by time alone
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
       mbar_init(&empty[s], 4);
     }
     *abort_flag = timed_out_before() ? 1 : 0;
+    *never_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -85,6 +87,7 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       const int row0 = b * p.C + s0;
+      int armed = 0;  // tiles whose loads were issued (stage t % kD8Stages)
       for (int t = 0; t < ntiles; ++t) {
         const int st = t % kD8Stages;
         if (t >= kD8Stages) {
@@ -93,12 +96,17 @@ __global__ void __launch_bounds__(kD8Threads, kD8CtasPerSm)
         uint8_t* kb = smem + st * kD8StageBytes;
         uint8_t* vb = kb + kD8KBytes;
         mbar_arrive_expect_tx(&full[st], kD8StageBytes);
+        ++armed;
         const int y = row0 + t * kD8TileKeys;
 #pragma unroll
         for (int c = 0; c < 3; ++c) tma_load_2d(kb + c * kD8BoxBytes, &tm_k, &full[st], g * 192 + c * 64, y);
 #pragma unroll
         for (int c = 0; c < 2; ++c) tma_load_2d(vb + c * kD8BoxBytes, &tm_v, &full[st], g * 128 + c * 64, y);
       }
+      // the CTA never exits with these copies in flight (after a timed-out
+      // wait the consumers may have stopped waiting for them)
+      for (int s = 0; s < kD8Stages; ++s)
+        drain_armed(&full[s], armed > s ? (armed - 1 - s) / kD8Stages + 1 : 0, never_flag);
     }
   } else {
     // ------------------------------------------------------------ consumers

@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   uint64_t* empty = full + kStages;
   uint64_t* q_full = empty + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(q_full + 1);
+  volatile int* never_flag = abort_flag + 1;  // never raised: bounds the drains by time alone
   uint8_t* sq = smem + kStages * kStageBytes + 128;  // [16 rows][kDecQRow] Q tile
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       mbar_init(&empty[s], 4);
     }
     mbar_init(q_full, 1);
+    *never_flag = 0;
     fence_mbar_init();
     // The G query rows of this KV head: one bulk copy per 384-byte row, into
     // rows kDecQRow apart (rows >= G are never read into a fragment).
@@ -149,8 +151,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
   // (the Q rows requested above land before the CTA leaves)
   if (*abort_flag) {
     if (threadIdx.x == 128) {
-      volatile int keep_waiting = 0;
-      wait_bounded(q_full, 0, &keep_waiting);
+      drain_armed(q_full, 1, never_flag);
     }
     return;
   }
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       const int row0 = b * p.C + s0;
+      int armed = 0;  // tiles whose loads were issued (stage t % kStages)
       for (int t = 0; t < ntiles; ++t) {
         const int st = t % kStages;
         if (t >= kStages) {
@@ -172,12 +174,18 @@ __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
         uint8_t* kb = smem + st * kStageBytes;
         uint8_t* vb = kb + 3 * kBox;
         mbar_arrive_expect_tx(&full[st], 5 * tile * 128);
+        ++armed;
         const int y = row0 + t * tile;
 #pragma unroll
         for (int c = 0; c < 3; ++c) tma_load_2d(kb + c * kBox, &tm_k, &full[st], g * 192 + c * 64, y);
 #pragma unroll
         for (int c = 0; c < 2; ++c) tma_load_2d(vb + c * kBox, &tm_v, &full[st], g * 128 + c * 64, y);
       }
+      // the CTA never exits with these copies in flight (after a timed-out
+      // wait the consumers may have stopped waiting for them)
+      for (int s = 0; s < kStages; ++s)
+        drain_armed(&full[s], armed > s ? (armed - 1 - s) / kStages + 1 : 0, never_flag);
+      drain_armed(q_full, 1, never_flag);
     }
   } else {
     // ------------------------------------------------------------ consumers

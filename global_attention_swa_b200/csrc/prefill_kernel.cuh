@@ -160,6 +160,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* o_empty = bars + 14; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+  uint64_t* mma_drain = bars + 18;  // teardown after a timed-out wait only
+  volatile int* never_flag = reinterpret_cast<volatile int*>(bars + 19);  // never raised
+  // for the teardown, kept here rather than in registers the loops carry: the
+  // phases the producer armed on q_full, on the K ring (tiles in order) and on
+  // v_full, and whether the MMA thread had work
+  int* armed = reinterpret_cast<int*>(bars + 20);  // [4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -177,6 +183,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       mbar_init(v_full, 1);
       mbar_init(v_empty, 1);
+      mbar_init(mma_drain, 1);
+      *never_flag = 0;
+      armed[0] = armed[1] = armed[2] = armed[3] = 0;
       // sampled once, so every thread of the CTA sees the same decision
       *abort_flag = timed_out_before() ? 1 : 0;
       fence_mbar_init();
@@ -226,6 +235,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int ks = kt & 1;
           if (kt >= 2 && !(ok = wait_bounded(&k_empty[ks], ((kt >> 1) - 1) & 1, abort_flag))) break;
           mbar_arrive_expect_tx(&k_full[ks], kPfKBytes);
+          armed[1] = kt + 1;
 #pragma unroll
           for (int c = 0; c < 3; ++c)
             tma_load_3d(smem + kPfOffK + ks * kPfKBytes + c * 16384, &tm_k, &k_full[ks], c * 64, it.g, row);
@@ -237,10 +247,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         ++n;
       }
+      // every item counted in n had its Q armed; V is armed for tiles [0, kt)
+      armed[0] = n;
+      armed[2] = kt;
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      armed[3] = rounds > 0;
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
       const uint32_t tS0 = tbase + 0, tS1 = tbase + 128, tO0 = tbase + 256, tO1 = tbase + 384;
@@ -505,6 +519,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // a role gave up: the loads and MMAs still in flight land before the CTA
+    // frees its TMEM and exits
+    if (warp == 8 && lane == 0) {
+      drain_armed(q_full, armed[0], never_flag);
+      drain_armed(&k_full[0], (armed[1] + 1) / 2, never_flag);
+      drain_armed(&k_full[1], armed[1] / 2, never_flag);
+      drain_armed(v_full, armed[2], never_flag);
+    }
+    if (warp == 9 && lane == 0 && armed[3]) drain_mma(mma_drain, never_flag);  // MMAs may have been issued
+    __syncthreads();
+  }
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);

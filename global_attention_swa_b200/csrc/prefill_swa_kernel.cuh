@@ -126,9 +126,13 @@ __global__ void __launch_bounds__(kSwThreads, 1)
   uint64_t* ml_empty = bars + 16; // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 19);
+  uint64_t* mma_drain = bars + 20;  // teardown after a timed-out wait only
+  volatile int* never_flag = reinterpret_cast<volatile int*>(bars + 21);  // never raised
   float4* ml = reinterpret_cast<float4*>(smem + kSwOffML);  // [2][128] (m, l, sink term) per row
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // phases the producer armed: Q for blocks 0, 1, ... (buffer n & 1), K and V per pair
+  int armed_q = 0, armed_k = 0, armed_v = 0;
   // the ones block, third 64-column block of the value operand: bf16 1.0
   for (int i = threadIdx.x; i < kSwKBox / 4; i += kSwThreads)
     reinterpret_cast<uint32_t*>(smem + kSwOffOnes)[i] = 0x3F803F80u;
@@ -149,6 +153,8 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       mbar_init(v_empty, 1);
       mbar_init(o_full, 1);
       mbar_init(o_empty, 128);
+      mbar_init(mma_drain, 1);
+      *never_flag = 0;
       *abort_flag = timed_out_before() ? 1 : 0;
       fence_mbar_init();
     }
@@ -172,6 +178,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
       tma_prefetch_desc(&tm_v);
       auto load_q = [&](const SwItem& it, int blk, int b) {
         mbar_arrive_expect_tx(&q_full[b], kSwQBytes);
+        ++armed_q;
 #pragma unroll
         for (int c = 0; c < 3; ++c)
           tma_load_3d(smem + kSwOffQ + b * kSwQBytes + c * 16384, &tm_q, &q_full[b], c * 64,
@@ -191,6 +198,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           if (blk == 0) {
             if (kp >= 1 && !(ok = wait_bounded(k_empty, (kp - 1) & 1, abort_flag))) break;
             mbar_arrive_expect_tx(k_full, 3 * N * 128);
+            ++armed_k;
 #pragma unroll
             for (int c = 0; c < 3; ++c)
               tma_load_3d(smem + kSwOffK + c * kSwKBox, &tm_k, k_full, c * 64, cur.g, cur.b0 + k0);
@@ -210,6 +218,7 @@ __global__ void __launch_bounds__(kSwThreads, 1)
           if (blk == 0) {
             if (kp >= 1 && !(ok = wait_bounded(v_empty, (kp - 1) & 1, abort_flag))) break;
             mbar_arrive_expect_tx(v_full, 2 * N * 128);
+            ++armed_v;
 #pragma unroll
             for (int c = 0; c < 2; ++c)
               tma_load_3d(smem + kSwOffV + c * kSwKBox, &tm_v, v_full, c * 64, cur.g, cur.b0 + k0);
@@ -456,6 +465,18 @@ __global__ void __launch_bounds__(kSwThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag) {
+    // a role gave up: the loads and MMAs still in flight land before the CTA
+    // frees its TMEM and exits
+    if (warp == 12 && lane == 0) {
+      drain_armed(&q_full[0], (armed_q + 1) / 2, never_flag);
+      drain_armed(&q_full[1], armed_q / 2, never_flag);
+      drain_armed(k_full, armed_k, never_flag);
+      drain_armed(v_full, armed_v, never_flag);
+    }
+    if (warp == 13 && lane == 0 && rounds > 0) drain_mma(mma_drain, never_flag);  // rounds > 0: MMAs may have been issued
+    __syncthreads();
+  }
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
