@@ -52,6 +52,7 @@ EXPORTED = (
     "mimo_attn_decode_merge",
     "mimo_attn_prefill_backward_workspace_size",
     "mimo_attn_prefill_backward",
+    "mimo_attn_wait_selftest",
     "mimo_attn_is_checked_build",
     "mimo_attn_checked_site",
     "mimo_attn_checked_selftest",
@@ -111,6 +112,8 @@ def _load():
     lib.mimo_attn_prefill_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
                                                vp, vp, vp, vp, vp, sz, vp]
     lib.mimo_attn_prefill_backward.restype = i32
+    lib.mimo_attn_wait_selftest.argtypes = [vp]
+    lib.mimo_attn_wait_selftest.restype = i32
     lib.mimo_attn_is_checked_build.argtypes = []
     lib.mimo_attn_is_checked_build.restype = i32
     lib.mimo_attn_checked_site.argtypes = [vp]
@@ -423,6 +426,15 @@ def mimo_attn_set_device_status(code, stream=None, device=None):
         stream.device if stream is not None else _current_device())
     with _on_device(dev):
         _check(lib.mimo_attn_set_device_status(int(code), _stream(stream, dev)))
+
+
+def mimo_attn_wait_selftest(stream=None, device=None):
+    """Failure-path test hook: a kernel whose wait runs out after its bound
+    (about 1 s) and records MIMO_ERR_TIMEOUT (see include/mimo_attn.h)."""
+    dev = torch.device(device) if device is not None else (
+        stream.device if stream is not None else _current_device())
+    with _on_device(dev):
+        _check(lib.mimo_attn_wait_selftest(_stream(stream, dev)))
 
 
 def mimo_attn_is_checked_build():

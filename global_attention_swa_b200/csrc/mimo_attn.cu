@@ -26,6 +26,35 @@
 #undef MIMO_FILE_ID
 #define MIMO_FILE_ID 10  // site numbers of the checked build
 
+namespace mimo {
+__device__ __align__(16) unsigned char g_wait_selftest_src[16];
+
+// A real time-out, for the failure-path test: one thread copies 16 bytes in
+// with a bulk copy; another waits on a barrier nothing ever arrives at, gives
+// up after the bound, records MIMO_ERR_TIMEOUT and raises the CTA's abort
+// flag; the teardown then waits for the armed copy, as the kernels do.
+__global__ void __launch_bounds__(64) wait_selftest_kernel() {
+  __shared__ __align__(16) unsigned char buf[16];
+  __shared__ __align__(8) uint64_t bars[2];  // [0] the copy, [1] never arrived at
+  __shared__ int abort_flag, never;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    abort_flag = 0;
+    never = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[0], 16);
+    bulk_load(buf, g_wait_selftest_src, 16, &bars[0]);
+  }
+  if (threadIdx.x == 32) wait_bounded(&bars[1], 0, &abort_flag);
+  __syncthreads();
+  if (*reinterpret_cast<volatile int*>(&abort_flag) && threadIdx.x == 0) drain_armed(&bars[0], 1, &never);
+}
+}  // namespace mimo
+
 #ifdef MIMO_CHECKED
 namespace mimo {
 // One row index past a 4-row buffer, checked and not used for any access.
@@ -785,6 +814,13 @@ int mimo_attn_checked_site(void* stream) {
       cuda_check(cudaMemcpyToSymbol(mimo::g_checked_site, &zero, sizeof(int)), "clear checked site"))
     return -1;
   return v;
+}
+
+mimo_status_t mimo_attn_wait_selftest(void* stream) {
+  mimo::wait_selftest_kernel<<<1, 64, 0, (cudaStream_t)stream>>>();
+  mimo_status_t st;
+  if ((st = cuda_check(cudaGetLastError(), "wait self-test launch"))) return st;
+  return ok();
 }
 
 mimo_status_t mimo_attn_checked_selftest(void* stream) {

@@ -1,12 +1,17 @@
 """Device-side failure reporting, tested without a failing GPU.
 
-Nothing here waits, faults or hangs: a timed-out wait is stood in for by
-pre-loading the device status word (mimo_attn_set_device_status), after which
-every kernel with bounded waits returns at entry; bad sequence metadata is
-caught by the kernels' own bounds checks before any access.  Each test checks
-the reported status, that nothing was written where nothing may be, and that
-the next call after the status is read runs normally.
+Nothing here faults or waits without a bound.  One real time-out runs: the
+library's self-test kernel waits about a second on a barrier that nothing
+arrives at, as a bounded wait would in a stuck pipeline, and records
+MIMO_ERR_TIMEOUT.  Elsewhere a timed-out wait is stood in for by pre-loading
+the device status word (mimo_attn_set_device_status), after which every kernel
+with bounded waits returns at entry; bad sequence metadata is caught by the
+kernels' own bounds checks before any access.  Each test checks the reported
+status, that nothing was written where nothing may be, and that the next call
+after the status is read runs normally.
 """
+
+import time
 
 import numpy as np
 import pytest
@@ -32,6 +37,23 @@ def expect_status(code):
         mimo.mimo_attn_device_status()
     assert ei.value.status == code, ei.value
     mimo.mimo_attn_device_status()  # read and cleared: OK now
+
+
+def test_a_wait_that_runs_out_records_timeout_and_the_next_calls_run():
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    mimo.mimo_attn_wait_selftest()
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert waited >= 0.9, waited  # it gave up at the bound, not before
+    expect_status(mimo.MIMO_ERR_TIMEOUT)
+    # the context still works: a decode after the time-out matches the oracle
+    x = W.decode_inputs([1, 300, 4000], 4096, 0, seed=9)
+    out, lse = mimo.mimo_attn_decode(x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda(),
+                                     0, x.sinks.cuda(), out_dtype=torch.float32)
+    mimo.mimo_attn_device_status()
+    ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, 0, x.sinks)
+    P.check(out, ro, lse, rl, what="decode after a time-out")
 
 
 def test_kernels_return_at_entry_after_a_recorded_timeout():
