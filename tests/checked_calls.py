@@ -60,6 +60,16 @@ def main():
         ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, window, x.sinks)
         P.check(out, ro, lse, rl, what=f"checked decode C={cap} W={window}")
 
+    # the decode entry point without a caller workspace (partials in the library's own array)
+    x = W.decode_inputs([1, 700, 5000, 0], 8192, 0, seed=21)
+    out = torch.empty((4, 64, 128), dtype=torch.float32, device="cuda")
+    lse = torch.empty((4, 64), dtype=torch.float32, device="cuda")
+    mimo.mimo_attn_decode_noalloc(x.q.cuda(), x.k_cache.cuda(), x.v_cache.cuda(), x.seqlens.cuda(), 0,
+                                  x.sinks.cuda(), out, lse)
+    clean("decode without workspace")
+    ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, 0, x.sinks)
+    P.check(out, ro, lse, rl, what="checked decode without workspace")
+
     # FP8 (e4m3) cache decode
     x = W.decode_inputs_fp8([1, 65, 1000, 129], 1024, 0, hq=8, hkv=2, seed=7)
     out, lse = mimo.mimo_attn_decode_fp8(x.q.cuda(), x.k_codes.cuda(), x.v_codes.cuda(), x.k_scale.cuda(),

@@ -53,6 +53,15 @@ def test_checked_runner_compiles():
     compile(open(path).read(), path, "exec")
 
 
+def test_wait_selftest_without_a_device_reports_a_cuda_error():
+    # no GPU here: the launch fails and the status says so (nothing waits)
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a device is present: the GPU test runs the real time-out")
+    assert mimo.lib.mimo_attn_wait_selftest(None) == mimo.MIMO_ERR_CUDA
+
+
 def test_selftest_is_refused_outside_the_checked_build():
     if mimo.CHECKED:
         pytest.skip("the checked build is loaded")
