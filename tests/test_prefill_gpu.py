@@ -205,6 +205,17 @@ def test_full_size_global_32k():
     full_size_check([32768], 0, per_seq_random=32, what="T=32768")
 
 
+def test_longest_position_swa():
+    """One sequence as long as the model's positions go (MiMoV2FlashConfig
+    max_position_embeddings = 131072) on the packed sliding-window kernel."""
+    full_size_check([131072], 129, per_seq_random=16, what="T=131072")
+
+
+def test_longest_position_global():
+    """The same length on a global layer: rows up to 131072 keys long."""
+    full_size_check([131072], 0, per_seq_random=4, what="T=131072")
+
+
 def test_full_size_varlen_stack():
     lengths = W.varlen_stack_lengths(0)
     sinks = W.stack_sinks(len(W.STACK_WINDOWS), seed=0)
