@@ -107,6 +107,19 @@ def test_ring_matches_linear_window():
     P.check(a, ro, la, rl, what="ring")
 
 
+@pytest.mark.parametrize("window", [0, 129])
+def test_full_caches(window):
+    """Sequences that fill their linear cache to the last slot (L == capacity),
+    and one slot short of it, under a multi-split plan."""
+    lengths = [65536, 65535, 1, 40000]
+    x = W.decode_inputs(lengths, 65536, window, seed=31 + window, device="cuda")
+    out, lse = mimo.mimo_attn_decode(x.q, x.k_cache, x.v_cache, x.seqlens, window, x.sinks,
+                                     out_dtype=torch.float32)
+    mimo.mimo_attn_device_status()
+    ro, rl = oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, window, x.sinks)
+    P.check(out, ro, lse, rl, what=f"full caches W={window}")
+
+
 def test_full_size_decode_global_and_ring():
     """Batch 64, lengths ~U[1024, 262144] in 262144-slot caches, and the 129-slot ring layer."""
     lengths = W.decode_b64_lengths(0)
