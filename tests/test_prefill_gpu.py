@@ -87,6 +87,19 @@ def test_per_head_kernel_varlen_every_length_class():
         P.check(out, ro, lse, rl, what=f"per-head varlen W={window}")
 
 
+@pytest.mark.parametrize("window", [0, 129])
+def test_many_short_sequences(window):
+    """A thousand sequences of 0 to 9 tokens in one pack (16 query heads on one
+    key/value head: the packed kernel for the window, the per-head kernel for
+    global): almost every work item starts a new sequence."""
+    rng = np.random.default_rng(71)
+    lengths = [int(L) for L in rng.integers(0, 10, 1000)]
+    x = W.prefill_inputs(lengths, hq=16, hkv=1, seed=72 + window)
+    out, lse = run_gpu(x, window, torch.float32)
+    ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens)
+    P.check(out, ro, lse, rl, what=f"1000 short sequences W={window}")
+
+
 def test_varlen_pack_equals_separate_calls():
     lengths = [200, 1, 513]
     x = W.prefill_inputs(lengths, hq=8, hkv=2, seed=5)
