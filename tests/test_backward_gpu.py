@@ -82,6 +82,16 @@ def test_model_heads_varlen_bf16(window):
 
 
 @pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
+def test_many_short_sequences(io):
+    """Three hundred sequences of 0 to 9 tokens: every key tile and query tile
+    is a sequence's first and last."""
+    lengths = [int(L) for L in np.random.default_rng(81).integers(0, 10, 300)]
+    got, ref = _run(lengths, 16, 1, 129, True, io, seed=82)
+    for name, a, b in zip(("dq", "dk", "dv", "dsinks"), got, ref):
+        grad_check(a, b, f"{name} short sequences")
+
+
+@pytest.mark.parametrize("io", [torch.float32, torch.bfloat16])
 def test_deterministic(io):
     a, _ = _run([200, 70], 16, 2, 129, True, io, seed=5)
     b, _ = _run([200, 70], 16, 2, 129, True, io, seed=5)
