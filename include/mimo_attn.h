@@ -336,6 +336,17 @@ mimo_status_t mimo_attn_device_status(void* stream);
 mimo_status_t mimo_attn_set_device_status(int code, void* stream);
 
 /*
+ * Failure-path test hook: launches one CTA in which a thread waits on a
+ * barrier that nothing arrives at.  The wait gives up after its bound (1 s),
+ * records MIMO_ERR_TIMEOUT in the device status word and raises the CTA's
+ * abort flag, and the CTA's teardown waits for the bulk copy another thread
+ * had in flight, as the library's kernels do after a timed-out wait.  Nothing
+ * faults and nothing waits without a bound.  Asynchronous on `stream`;
+ * mimo_attn_device_status() then reports MIMO_ERR_TIMEOUT (and clears it).
+ */
+mimo_status_t mimo_attn_wait_selftest(void* stream);
+
+/*
  * Bounds-checked build.  The same sources compiled with -DMIMO_CHECKED give
  * libmimo_attn_checked.so: every kernel checks each row index it forms for a
  * global read or write against the row count of that buffer before the
@@ -354,17 +365,6 @@ mimo_status_t mimo_attn_set_device_status(int code, void* stream);
  *   memory, so that the status word then holds MIMO_ERR_BOUNDS and the site
  *   is set; asynchronous on `stream`.
  */
-/*
- * Failure-path test hook: launches one CTA in which a thread waits on a
- * barrier that nothing arrives at.  The wait gives up after its bound (1 s),
- * records MIMO_ERR_TIMEOUT in the device status word and raises the CTA's
- * abort flag, and the CTA's teardown waits for the bulk copy another thread
- * had in flight, as the library's kernels do after a timed-out wait.  Nothing
- * faults and nothing waits without a bound.  Asynchronous on `stream`;
- * mimo_attn_device_status() then reports MIMO_ERR_TIMEOUT (and clears it).
- */
-mimo_status_t mimo_attn_wait_selftest(void* stream);
-
 int mimo_attn_is_checked_build(void);
 int mimo_attn_checked_site(void* stream);
 mimo_status_t mimo_attn_checked_selftest(void* stream);
