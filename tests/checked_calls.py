@@ -112,6 +112,23 @@ def main():
             clean(f"backward W={window} {odt}")
             assert all(torch.isfinite(t).all() for t in grads if t is not None)
 
+    # the bench's full-size workloads: no row index of any kernel may leave its
+    # buffer at these sizes either (results are checked by the parity tests)
+    for window in (129, 0):
+        x = W.prefill_inputs([32768], seed=40 + window, device="cuda")
+        out, lse = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, 32768)
+        clean(f"full-size prefill W={window}")
+        assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+        del x, out, lse
+    lengths = W.decode_b64_lengths(0)
+    for cap, window in ((W.DECODE_GA_CAPACITY, 0), (129, 129)):
+        x = W.decode_inputs(lengths, cap, window, seed=42, device="cuda")
+        out, lse = mimo.mimo_attn_decode(x.q, x.k_cache, x.v_cache, x.seqlens, window, x.sinks)
+        clean(f"full-size decode C={cap}")
+        assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+        del x, out, lse
+    torch.cuda.empty_cache()
+
     # the self-test: a failing check that touches no memory
     mimo.mimo_attn_checked_selftest()
     st = mimo.lib.mimo_attn_device_status(None)
