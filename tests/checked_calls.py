@@ -112,14 +112,22 @@ def main():
             clean(f"backward W={window} {odt}")
             assert all(torch.isfinite(t).all() for t in grads if t is not None)
 
-    # the bench's full-size workloads: no row index of any kernel may leave its
-    # buffer at these sizes either (results are checked by the parity tests)
+    # the bench's full-size workloads (and its backward case): no row index of
+    # any kernel may leave its buffer at these sizes either (results are checked
+    # by the parity tests)
     for window in (129, 0):
         x = W.prefill_inputs([32768], seed=40 + window, device="cuda")
         out, lse = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, window, x.cu_seqlens, 32768)
         clean(f"full-size prefill W={window}")
         assert torch.isfinite(out).all() and torch.isfinite(lse).all()
         del x, out, lse
+    x = W.prefill_inputs([8192], seed=43, device="cuda")
+    out, lse = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, 0, x.cu_seqlens, 8192)
+    dout = torch.randn(out.shape, device="cuda").to(out.dtype)
+    grads = mimo.mimo_attn_prefill_backward(x.q, x.k, x.v, out, lse, dout, x.sinks, 0, x.cu_seqlens, 8192)
+    clean("full-size backward T=8192")
+    assert all(torch.isfinite(t).all() for t in grads)
+    del x, out, lse, dout, grads
     lengths = W.decode_b64_lengths(0)
     for cap, window in ((W.DECODE_GA_CAPACITY, 0), (129, 129)):
         x = W.decode_inputs(lengths, cap, window, seed=42, device="cuda")
