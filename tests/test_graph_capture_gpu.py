@@ -1,0 +1,95 @@
+"""The entry points run inside a captured CUDA graph.
+
+A serving loop captures a decode step once and replays it every token with
+new inputs copied into the captured buffers; a training or prefill loop can
+do the same for fixed shapes.  None of the calls synchronises the host or
+allocates device memory when its buffers are given, so each is captured as
+its kernel launches.  Each test captures the calls, replays the graph with
+two different sets of inputs, and compares every replay with the oracle.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests import parity_util as P
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import global_attention_swa_b200 as mimo
+
+
+def _capture(fn):
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # first calls outside the capture (one-time host setup)
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def test_decode_step_replays():
+    lengths = [1, 700, 5000, 129]
+    ga = W.decode_inputs(lengths, 8192, 0, seed=41, device="cuda")        # several splits + combine
+    sw = W.decode_inputs(lengths, 129, 129, seed=42, device="cuda")       # 129-slot ring
+    ws = torch.empty(max(1, mimo.mimo_attn_decode_workspace_size(64, 4, 4, 8192, 0)),
+                     dtype=torch.uint8, device="cuda")
+    o_ga = torch.empty((4, 64, 128), dtype=torch.float32, device="cuda")
+    l_ga = torch.empty((4, 64), dtype=torch.float32, device="cuda")
+    o_sw, l_sw = torch.empty_like(o_ga), torch.empty_like(l_ga)
+
+    def step():
+        mimo.mimo_attn_decode(ga.q, ga.k_cache, ga.v_cache, ga.seqlens, 0, ga.sinks,
+                              out=o_ga, lse=l_ga, workspace=ws)
+        mimo.mimo_attn_decode(sw.q, sw.k_cache, sw.v_cache, sw.seqlens, 129, sw.sinks,
+                              out=o_sw, lse=l_sw)
+
+    g = _capture(step)
+    gen = torch.Generator(device="cuda").manual_seed(43)
+    for trial in range(2):
+        ga.q.copy_(torch.randn(ga.q.shape, generator=gen, device="cuda").to(ga.q.dtype))
+        sw.q.copy_(torch.randn(sw.q.shape, generator=gen, device="cuda").to(sw.q.dtype))
+        o_ga.fill_(float("nan"))
+        o_sw.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        mimo.mimo_attn_device_status()
+        ro, rl = oracle.decode(ga.q, ga.k_cache, ga.v_cache, ga.seqlens, 0, ga.sinks)
+        P.check(o_ga, ro, l_ga, rl, what=f"graph replay {trial}: global decode")
+        ro, rl = oracle.decode(sw.q, sw.k_cache, sw.v_cache, sw.seqlens, 129, sw.sinks)
+        P.check(o_sw, ro, l_sw, rl, what=f"graph replay {trial}: ring decode")
+    del g
+
+
+def test_prefill_replays():
+    lengths = [300, 1, 129, 0, 513]
+    x = W.prefill_inputs(lengths, seed=44, device="cuda")
+    nt = sum(lengths)
+    outs = {w: (torch.empty((nt, 64, 128), dtype=torch.float32, device="cuda"),
+                torch.empty((64, nt), dtype=torch.float32, device="cuda")) for w in (129, 0)}
+
+    def step():
+        for w, (o, l) in outs.items():
+            mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, w, x.cu_seqlens, max(lengths), out=o, lse=l)
+
+    g = _capture(step)
+    gen = torch.Generator(device="cuda").manual_seed(45)
+    for trial in range(2):
+        for t in (x.q, x.k, x.v):
+            t.copy_(torch.randn(t.shape, generator=gen, device="cuda").to(t.dtype))
+        for o, _ in outs.values():
+            o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        mimo.mimo_attn_device_status()
+        for w, (o, l) in outs.items():
+            ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, w, x.cu_seqlens)
+            P.check(o, ro, l, rl, what=f"graph replay {trial}: prefill W={w}")
+    del g
