@@ -1,4 +1,4 @@
-"""The entry points run inside a captured CUDA graph.
+"""The entry points run inside a captured CUDA graph (decode, prefill, backward).
 
 A serving loop captures a decode step once and replays it every token with
 new inputs copied into the captured buffers; a training or prefill loop can
@@ -92,4 +92,36 @@ def test_prefill_replays():
         for w, (o, l) in outs.items():
             ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, w, x.cu_seqlens)
             P.check(o, ro, l, rl, what=f"graph replay {trial}: prefill W={w}")
+    del g
+
+
+def test_backward_replays():
+    lengths = [200, 0, 129]
+    x = W.prefill_inputs(lengths, hq=16, hkv=1, seed=46, device="cuda")
+    nt = sum(lengths)
+    out = torch.empty((nt, 16, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((16, nt), dtype=torch.float32, device="cuda")
+    dout = torch.empty_like(out)
+    res = {}
+
+    def step():
+        mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, 0, x.cu_seqlens, 200, out=out, lse=lse)
+        res["g"] = mimo.mimo_attn_prefill_backward(x.q, x.k, x.v, out, lse, dout, x.sinks, 0,
+                                                   x.cu_seqlens, 200)
+
+    from oracle.backward import prefill_backward
+
+    gen = torch.Generator(device="cuda").manual_seed(47)
+    dout.copy_(torch.randn(dout.shape, generator=gen, device="cuda").to(dout.dtype))
+    g = _capture(step)
+    for trial in range(2):
+        for t in (x.q, x.k, x.v, dout):
+            t.copy_(torch.randn(t.shape, generator=gen, device="cuda").to(t.dtype))
+        g.replay()
+        torch.cuda.synchronize()
+        mimo.mimo_attn_device_status()
+        ref = prefill_backward(x.q, x.k, x.v, dout, x.sinks, 0, x.cu_seqlens)
+        for name, a, b in zip(("dq", "dk", "dv", "dsinks"), res["g"], ref):
+            err = np.abs(P.to64(a) - b).max()
+            assert err <= 1e-2 * np.abs(b).max() + 1e-4, f"graph replay {trial}: {name} {err:.3e}"
     del g
