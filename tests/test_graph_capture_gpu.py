@@ -125,3 +125,25 @@ def test_backward_replays():
             err = np.abs(P.to64(a) - b).max()
             assert err <= 1e-2 * np.abs(b).max() + 1e-4, f"graph replay {trial}: {name} {err:.3e}"
     del g
+
+
+def test_calls_on_two_streams_at_once():
+    """A prefill on one stream and a decode on another, launched back to back
+    so that they can run concurrently: each result matches the oracle."""
+    x = W.prefill_inputs([700, 129], seed=48, device="cuda")
+    d = W.decode_inputs([1, 3000, 129], 4096, 0, seed=49, device="cuda")
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    s1.wait_stream(torch.cuda.current_stream())
+    s2.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s1):
+        po, pl = mimo.mimo_attn_prefill(x.q, x.k, x.v, x.sinks, 129, x.cu_seqlens, 700,
+                                        out_dtype=torch.float32, stream=s1)
+    with torch.cuda.stream(s2):
+        do, dl = mimo.mimo_attn_decode(d.q, d.k_cache, d.v_cache, d.seqlens, 0, d.sinks,
+                                       out_dtype=torch.float32, stream=s2)
+    torch.cuda.synchronize()
+    mimo.mimo_attn_device_status()
+    ro, rl = oracle.prefill(x.q, x.k, x.v, x.sinks, 129, x.cu_seqlens)
+    P.check(po, ro, pl, rl, what="prefill on its own stream")
+    ro, rl = oracle.decode(d.q, d.k_cache, d.v_cache, d.seqlens, 0, d.sinks)
+    P.check(do, ro, dl, rl, what="decode on its own stream")
