@@ -345,6 +345,65 @@ def test_every_wrapper_accepts_its_documented_dtypes(monkeypatch):
             "mimo_attn_rope_append", "mimo_attn_decode_merge", "mimo_attn_decode_noalloc"} <= set(seen)
 
 
+def test_a_failed_launch_reaches_the_caller_as_an_exception(monkeypatch):
+    """A launch failure inside the library (simulated: a stand-in library whose
+    entry points return MIMO_ERR_CUDA, as the real one does when
+    cudaGetLastError reports one) reaches the caller of every wrapper as
+    MimoAttnError carrying the status and the library's message."""
+    import types
+
+    import torch
+
+    class FailingLib:
+        def mimo_attn_last_error(self):
+            return b"prefill launch: unspecified launch failure"
+
+        def mimo_attn_decode_workspace_size(self, *a):
+            return 1024
+
+        def mimo_attn_decode_fp8_workspace_size(self, *a):
+            return 1024
+
+        def mimo_attn_prefill_backward_workspace_size(self, *a):
+            return 1024
+
+        def __getattr__(self, name):
+            return lambda *a: mimo.MIMO_ERR_CUDA
+
+    real_ptr = mimo._ptr
+
+    def host_ptr(t, name="tensor", dtype=None):
+        if t is None:
+            return None
+        proxy = types.SimpleNamespace(is_cuda=True, is_contiguous=t.is_contiguous, dtype=t.dtype,
+                                      data_ptr=t.data_ptr)
+        return real_ptr(proxy, name, dtype)
+
+    monkeypatch.setattr(mimo, "lib", FailingLib())
+    monkeypatch.setattr(mimo, "_ptr", host_ptr)
+    monkeypatch.setattr(mimo, "_stream", lambda stream, dev: None)
+    bf, f32, i32 = torch.bfloat16, torch.float32, torch.int32
+    q = torch.zeros((24, 4, 192), dtype=bf)
+    k = torch.zeros((24, 1, 192), dtype=bf)
+    v = torch.zeros((24, 1, 128), dtype=bf)
+    cu = torch.tensor([0, 24], dtype=i32)
+    qd = torch.zeros((2, 4, 192), dtype=bf)
+    kc = torch.zeros((2, 16, 1, 192), dtype=bf)
+    vc = torch.zeros((2, 16, 1, 128), dtype=bf)
+    sl = torch.tensor([3, 16], dtype=i32)
+    calls = [
+        lambda: mimo.mimo_attn_prefill(q, k, v, None, 129, cu, 24),
+        lambda: mimo.mimo_attn_decode(qd, kc, vc, sl, 0, None),
+        lambda: mimo.mimo_attn_decode_merge(torch.zeros((2, 2, 4, 128)), torch.zeros((2, 2, 4)), None),
+        lambda: mimo.mimo_attn_device_status(device="cpu"),
+    ]
+    for call in calls:
+        with pytest.raises(mimo.MimoAttnError) as e:
+            call()
+        assert e.value.status == mimo.MIMO_ERR_CUDA
+        assert "launch failure" in str(e.value)
+
+
 def test_binding_refuses_a_stream_of_another_device():
     """A caller's stream must belong to the device the tensors live on."""
     import types
